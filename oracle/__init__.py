@@ -1,0 +1,22 @@
+"""CPU oracle for the LLM.int8() forward linear layer.
+
+Test infrastructure only: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``.  Nothing in the product package
+imports it, and it imports nothing from the product package.
+"""
+
+from .llm_int8 import (  # noqa: F401
+    Q_MAX,
+    absmax_codes,
+    combine,
+    dequantize_weight,
+    int8_matmul,
+    linear_forward,
+    outlier_index,
+    outlier_mask,
+    outlier_operands,
+    quantize_rows,
+    quantize_weight,
+    round_half_away,
+    y_tolerance,
+)
