@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Throughput of the LLM.int8() forward linear layer on B200.
+
+One step = one full forward (outlier columns, row quantisation + gathers, the
+int8 tensor-core product with the fused fp16 outlier product and epilogue) over
+one batch of seeded synthetic input already resident in HBM.  The default
+workload is BLOOM-176B's FFN-up projection at prefill: X fp16 [8192, 14336]
+with 8 outlier feature dimensions, W [57344, 14336] quantised to int8 CB/SCB.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                        [--impl ours|reference]
+Under torchrun (N > 1) every rank runs an independent problem of the same
+shape (weak scaling; no data-path collective); the reported time is the max
+over ranks and the value is the work of all ranks divided by it.
+``--impl reference`` times the CPU oracle (a deliberately plain numpy
+restatement of the method) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int8_mixed_precision_column_b200 import workloads  # noqa: E402
+
+METRIC = "int8-decomposed linear TOPS & tokens/s at BLOOM shapes; % of int8 TC peak / HBM"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 POPS)
+
+WORKLOADS = {
+    "bloom176b_ffn_up_prefill": lambda dev, seed: workloads.bloom_ffn_up_prefill(8192, seed=seed, device=dev),
+    "llama7b_prefill": lambda dev, seed: workloads.llama7b_prefill(seed=seed, device=dev),
+    "bloom176b_ffn_up_decode_T1": lambda dev, seed: workloads.bloom_ffn_up_decode(1, seed=seed, device=dev),
+    "bloom176b_ffn_up_decode_T4": lambda dev, seed: workloads.bloom_ffn_up_decode(4, seed=seed, device=dev),
+    "bloom176b_ffn_up_decode_T16": lambda dev, seed: workloads.bloom_ffn_up_decode(16, seed=seed, device=dev),
+    "density_sweep_nout512": lambda dev, seed: workloads.density_sweep(512, seed=seed, device=dev),
+}
+DEFAULT_WORKLOAD = "bloom176b_ffn_up_prefill"
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def load_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env() -> tuple[int, int, int]:
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def reduce_max(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def algorithmic_work(T: int, K: int, N: int, n_out: int) -> dict:
+    """Ops and bytes one forward must do, independent of the implementation."""
+    return {
+        "int8_ops": 2.0 * T * N * K,
+        "fp16_flops": 2.0 * T * N * n_out,
+        # HBM bytes of the product kernel: CB once, X codes once, Y once, scales, bias
+        "product_bytes": float(N * K + T * K + 2 * T * N + 4 * N + 2 * N + 4 * T + 2 * T * n_out
+                               + 2 * N * n_out),
+    }
+
+
+def pci_bus_id(dev) -> str | None:
+    """nvidia-smi style bus id ("00000000:1B:00.0") of a torch device, if torch exposes it."""
+    pr = torch.cuda.get_device_properties(dev)
+    try:
+        return f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+    except AttributeError:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling during the timed region (rank 0's GPU)."""
+
+    FIELDS = ("timestamp,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = (bus_id or "").lower()
+        self.proc = None
+        self.path = None
+        self.t0 = self.t1 = 0.0
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        mine = [r for r in rows if self.bus_id and r[1].lower()[-12:] == self.bus_id[-12:]] or rows
+
+        def ts(r):
+            try:
+                return time.mktime(time.strptime(r[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+            except ValueError:
+                return None
+
+        window = [r for r in mine if ts(r) is not None and self.t0 - 1.0 <= ts(r) <= self.t1 + 1.0] or mine
+        sm = [float(r[2]) for r in window if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in window if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in window for n, v in zip(names, r[6:10]) if v.lower() == "active"})
+        pw = [float(r[4]) for r in window if r[4].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(window), "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank) -> dict | None:
+    from int8_mixed_precision_column_b200 import build, native
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build.build()
+    native.lib()
+    p = WORKLOADS[args.workload]("cuda", rank)
+    T, K, N = p.T, p.K, p.N
+    bias = p.bias
+    CB, SCB = native.int8_quantize_weight(p.W)
+    cpu_sample = sample_problem(p, 256, 4096) if (world == 1 and not args.no_cpu_baseline) else None
+    del p.W
+    torch.cuda.empty_cache()
+    X = p.X
+    Y = torch.empty((T, N), dtype=torch.float16, device=dev)
+    idx = torch.empty((K,), dtype=torch.int32, device=dev)
+    n_out = torch.empty((1,), dtype=torch.int32, device=dev)
+    ws = native.new_workspace(T, K, N, dev)
+    working_set = T * K * 3 + N * K + T * N * 2
+    flush = working_set < 2 * L2_BYTES
+    scrub = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
+
+    nsteps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nsteps + args.warmup)]
+    for row in ev:
+        for e in row:
+            e.record()
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def step(i):
+        native.int8_linear_forward_timed(X, CB, SCB, bias, p.threshold, Y, idx, n_out, ws, ev[i])
+
+    for i in range(args.warmup):
+        if flush:
+            scrub.add_(1)
+        step(nsteps + i)
+    torch.cuda.synchronize()
+    st, where = native.int8_check_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {native.int8_status_string(st)} at {where:#x}")
+    n_outliers = int(n_out.item())
+
+    sampler = ClockSampler(pci_bus_id(dev))
+    if rank == 0:
+        sampler.start()
+        time.sleep(1.0)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.mark_begin()
+    outer[0].record()
+    for i in range(nsteps):
+        if flush:
+            scrub.add_(1)
+        step(i)
+    outer[1].record()
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    barrier(world)
+    clocks = sampler.stop() if rank == 0 else None
+
+    st, where = native.int8_check_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {native.int8_status_string(st)} at {where:#x}")
+    step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(nsteps)]
+    prod_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(nsteps)]
+    outl_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(nsteps)]
+    rowq_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(nsteps)]
+    total_ms = outer[0].elapsed_time(outer[1]) if not flush else sum(step_ms)
+    ms_per_step = reduce_max(total_ms / nsteps, world, dev)
+
+    # end to end through the host-buffer entry point: pinned X in, Y/idx/n_out out, per step
+    e2e = None
+    if not args.no_e2e:
+        Xh = X.cpu().pin_memory()
+        Yh = torch.empty((T, N), dtype=torch.float16).pin_memory()
+        idx_h = torch.empty((K,), dtype=torch.int32).pin_memory()
+        n_h = torch.empty((1,), dtype=torch.int32).pin_memory()
+        del ws
+        torch.cuda.empty_cache()
+        wsh = torch.empty(native.int8_linear_forward_host_workspace_bytes(T, K, N), dtype=torch.uint8, device=dev)
+        for _ in range(min(args.warmup, 3)):
+            native.int8_linear_forward_host(Xh, CB, SCB, bias, p.threshold, Yh, wsh, idx_h, n_h)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ne = max(3, min(nsteps, 20))
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(ne):
+            native.int8_linear_forward_host(Xh, CB, SCB, bias, p.threshold, Yh, wsh, idx_h, n_h)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = reduce_max(e0.elapsed_time(e1) / ne, world, dev)
+        e2e = {"value": 2.0 * T * N * K * world / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+               "ms_per_step": e2e_ms, "steps": ne,
+               "h2d_bytes_per_step": T * K * 2,
+               "d2h_bytes_per_step": T * N * 2 + K * 4 + 4 + 64,
+               "api": "int8_linear_forward_host (pinned host X/Y, resident CB/SCB)"}
+
+    if rank != 0:
+        return None
+    work = algorithmic_work(T, K, N, n_outliers)
+    peaks, peak_src = load_peaks()
+    prod_avg = statistics.mean(prod_ms)
+    decode = T <= 16
+    if decode:
+        achieved = work["product_bytes"] / (prod_avg * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "gemv_i8_decode_kernel",
+                "peak_source": f"{peak_src} hbm_gbs (copy)",
+                "algorithmic_bytes_per_launch": work["product_bytes"], "ms_per_launch": prod_avg}
+    else:
+        peak = peaks["bf16_tflops"] * INT8_PER_BF16
+        achieved = work["int8_ops"] / (prod_avg * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS",
+                "frac": achieved / peak, "traffic": None, "kernel": "gemm_i8_tc_kernel",
+                "peak_source": f"{peak_src} bf16_tflops (burst) x {INT8_PER_BF16} nominal int8:bf16 ratio",
+                "algorithmic_ops_per_launch": work["int8_ops"], "ms_per_launch": prod_avg}
+    launches_per_step = 3 if p.threshold > 0 else 2
+    out = {
+        "metric": METRIC,
+        "value": work["int8_ops"] * world / (ms_per_step * 1e-3) / 1e12,
+        "unit": "TOPS",
+        "tokens_per_s": T * world / (ms_per_step * 1e-3),
+        "n_gpus": world,
+        "steps": nsteps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8 x int8 -> int32 (+ fp16 outlier product, fp32 accumulate), fp16 in/out",
+        "data": "synthetic (seeded; X ~ N(0,1) with planted outlier columns, W ~ N(0, 0.02^2))",
+        "config": {"workload": args.workload, "T": T, "K": K, "N": N, "threshold": p.threshold,
+                   "n_out": n_outliers, "parallelism": f"independent problem per rank x{world}",
+                   "l2": "L2 flushed between steps" if flush else "inputs larger than L2 (no flush)"},
+        "stage_ms": {"outliers": statistics.mean(outl_ms), "rowquant": statistics.mean(rowq_ms),
+                     "product": prod_avg},
+        "roofline": roof,
+        "gpu_launches": launches_per_step * nsteps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "device": torch.cuda.get_device_name(dev),
+    }
+    if cpu_sample is not None:
+        out["cpu_baseline"] = cpu_baseline(cpu_sample, p.threshold, seconds=args.cpu_seconds)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline / reference arm
+# ---------------------------------------------------------------------------
+
+def sample_problem(p, rows: int, cols: int):
+    """A sub-problem of the workload: `rows` token rows x `cols` output features."""
+    gen = np.random.default_rng(1234)
+    T, N = p.T, p.N
+    r = np.sort(gen.choice(T, size=min(rows, T), replace=False))
+    c = np.sort(gen.choice(N, size=min(cols, N), replace=False))
+    X = p.X[torch.as_tensor(r, device=p.X.device)].cpu().numpy()
+    W = p.W[torch.as_tensor(c, device=p.W.device)].cpu().numpy()
+    b = None if p.bias is None else p.bias[torch.as_tensor(c, device=p.bias.device)].cpu().numpy()
+    return X, W, b
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_rate(X, W, b, thr, seconds: float) -> tuple[float, int, float]:
+    """Run the oracle forward on (X, W) repeatedly for ~`seconds`; returns (TOPS, reps, s/rep)."""
+    from oracle import llm_int8 as O
+
+    CB, SCB = O.quantize_weight(W)  # layer set-up, not part of a step
+    T, K = X.shape
+    N = W.shape[0]
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        O.linear_forward(X, CB, SCB, b, thr)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return 2.0 * T * N * K * reps / el / 1e12, reps, el / reps
+
+
+def cpu_baseline(sample, threshold: float, seconds: float = 12.0) -> dict:
+    X, W, b = sample
+    v, reps, per = oracle_rate(X, W, b, threshold, seconds)
+    return {"value": v, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"full oracle forward on {X.shape[0]} token rows x {W.shape[0]} output features of the "
+                      f"workload (K={X.shape[1]}), repeated {reps}x ({per:.2f} s each)"}
+
+
+def run_reference(args, rank, world, local_rank) -> dict | None:
+    if rank != 0:
+        return None
+    p = WORKLOADS[args.workload]("cpu", 0)
+    T, K, N = p.T, p.K, p.N
+    X, W, b = sample_problem(p, rows=64, cols=2048)
+    from oracle import llm_int8 as O
+
+    CB, SCB = O.quantize_weight(W)
+    for _ in range(args.warmup):
+        O.linear_forward(X, CB, SCB, b, p.threshold)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.linear_forward(X, CB, SCB, b, p.threshold)
+    el = time.perf_counter() - t0
+    ms = el / args.steps * 1e3
+    ops = 2.0 * X.shape[0] * W.shape[0] * K
+    v = ops / (ms * 1e-3) / 1e12
+    sample = (f"oracle forward on {X.shape[0]} token rows x {W.shape[0]} output features of the workload "
+              f"(T={T}, K={K}, N={N}) per step")
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TOPS",
+            "tokens_per_s": X.shape[0] / (ms * 1e-3), "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8 codes, fp64 reference arithmetic (numpy)",
+            "data": "synthetic (seeded)",
+            "config": {"workload": args.workload, "T": T, "K": K, "N": N, "threshold": p.threshold},
+            "cpu_baseline": {"value": v, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        out = run_reference(args, rank, world, local_rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,190 @@
+/*
+ * int8mp.h -- C ABI of libint8mp, the LLM.int8() forward linear layer
+ * (bitsandbytes Linear8bitLt with has_fp16_weights=False) for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation (Hugging Face integration page for LLM.int8(), "Core idea of
+ * LLM.int8()", steps 1-3, and "Quantization mechanics"):
+ *   1. outlier columns: k is an outlier if |X[t,k]| > threshold for some token t
+ *      (bitsandbytes Linear8bitLt docstring, `threshold`; issue #1609: the
+ *      threshold acts on activations; state.idx lists the outlier columns);
+ *   2. the non-outlier part of X is quantised row-wise to int8 with scale
+ *      127/absmax (absmax over the row's non-outlier columns), the weight
+ *      row-wise per output feature (CB int8, SCB = absmax fp32, so that W is
+ *      recovered as CB*SCB/127, "Integration into transformers"); the two are
+ *      multiplied in int8 with int32 accumulation, while the outlier columns
+ *      are multiplied in 16-bit floating point;
+ *   3. the int8 result is dequantised with (row scale) x (column scale) / 127^2,
+ *      summed with the 16-bit result and the bias, and returned in fp16.
+ *
+ * Conventions for every entry point:
+ *   - Matrices are row-major.  X fp16 [T,K] (K = in_features contiguous),
+ *     W fp16 [N,K] (the nn.Linear weight layout, N = out_features),
+ *     Y fp16 [T,N].
+ *   - Pointers documented as "device" must be CUDA device memory of the
+ *     current device; the caller owns every buffer.  The library allocates
+ *     nothing and keeps no per-call state outside the caller's workspace.
+ *   - Calls are asynchronous on `stream` unless stated otherwise.  Argument
+ *     errors are reported synchronously before any work is enqueued; launch
+ *     failures are reported as I8_ERR_CUDA.  A device-side wait that gives up
+ *     (I8_ERR_TIMEOUT) is recorded in the workspace and read back by
+ *     int8_check_status().
+ *   - Shape rules: K and N are positive multiples of 16 with K <= 131072
+ *     (so that |acc| <= K*127^2 fits int32); T >= 0.  X, CB, Y and the
+ *     workspace must be 16-byte aligned, SCB 4-byte aligned, bias and idx
+ *     naturally aligned.
+ *   - Results are deterministic: idx is ascending, and the integer stages
+ *     (idx, n_out, CB, SCB, the int8 codes of X, the row scales and the int32
+ *     accumulators) are identical from run to run.
+ */
+#ifndef INT8MP_H_
+#define INT8MP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum i8_status {
+  I8_OK = 0,
+  I8_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad shape */
+  I8_ERR_WORKSPACE = 2,   /* workspace too small or misaligned */
+  I8_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  I8_ERR_TIMEOUT = 4,     /* a device-side wait gave up; the kernel returned early */
+  I8_ERR_UNSUPPORTED = 5  /* no sm_100 device, or the driver lacks TMA map encoding */
+} i8_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* int8_status_string(int status);
+
+/* Library ABI version (major*100 + minor). */
+int int8_version(void);
+
+/*
+ * Weight quantisation, done once per layer (the `.to(device)` step of
+ * Linear8bitLt with has_fp16_weights=False; Hugging Face integration page,
+ * "Integration into transformers": CB in [-127, 127], W ~ CB*SCB/127).
+ *   W   device fp16 [N,K]   input weight, read only
+ *   CB  device int8 [N,K]   output codes: clamp(roundf(W*(127/SCB[j])), -127, 127),
+ *                           ties away from zero; all zero when SCB[j] == 0
+ *   SCB device fp32 [N]     output per-row absmax max_k |W[j,k]|
+ * Asynchronous on `stream`.
+ */
+i8_status int8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* CB, float* SCB,
+                               cudaStream_t stream);
+
+/* Bytes of device workspace int8_linear_forward needs for a T x K -> N
+ * forward (worst case: every column an outlier).  Host-only; never fails. */
+size_t int8_linear_workspace_bytes(int64_t T, int64_t K, int64_t N);
+
+/*
+ * The forward (steps 1-3 above).
+ *   X         device fp16 [T,K]   activations, read only
+ *   CB, SCB   device              output of int8_quantize_weight for [N,K]
+ *   bias      device fp16 [N] or NULL (no bias)
+ *   threshold outlier threshold; a column is an outlier iff some |X[t,k]| >
+ *             threshold (strict).  threshold <= 0 or NaN switches the
+ *             decomposition off (no outlier columns, pure int8 product).
+ *             NaN entries of X never flag a column.
+ *   Y         device fp16 [T,N]   output
+ *   idx       device int32 [K]    capacity K; receives the ascending outlier
+ *                                 column indices (Linear8bitLt state.idx)
+ *   n_out     device int32 [1]    receives the number of outlier columns
+ *   workspace device, >= int8_linear_workspace_bytes(T,K,N) bytes, 256-byte
+ *             aligned; its contents need no initialisation and are
+ *             overwritten.  One workspace must not be shared by forwards
+ *             that can run concurrently.
+ * T <= 16 takes the weight-streaming decode kernel, larger T the tensor-core
+ * GEMM; both give the same integer stages.  Asynchronous on `stream`; n_out
+ * stays on the device (no host synchronisation).
+ */
+i8_status int8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                              const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
+                              int32_t* n_out, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/* As int8_linear_forward, with the product kernel chosen explicitly:
+ * path 0 = automatic (as above), 1 = tensor-core GEMM (any T),
+ * 2 = decode GEMV (T <= 16, else I8_ERR_INVALID_ARG). */
+i8_status int8_linear_forward_path(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                                   const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
+                                   int32_t* n_out, void* workspace, size_t workspace_bytes, int path,
+                                   cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of
+ * `workspace`: I8_OK, or I8_ERR_TIMEOUT if a kernel of the most recent
+ * forward using this workspace gave up a wait.  *where (may be NULL)
+ * receives the tag of the wait that gave up.
+ */
+i8_status int8_check_status(void* workspace, uint32_t* where, cudaStream_t stream);
+
+/*
+ * The forward with HOST activations and output: copies X host->device,
+ * runs int8_linear_forward, copies Y (and idx, n_out when non-NULL) back,
+ * and synchronises `stream` before returning (blocking).  CB, SCB, bias stay
+ * device pointers (the quantised layer is resident).  X_host and Y_host
+ * should be page-locked for full copy bandwidth.
+ *   idx_host  host int32 [K] or NULL;  n_out_host host int32 [1] or NULL.
+ *   workspace device, >= int8_linear_forward_host_workspace_bytes(T,K,N).
+ * Returns I8_ERR_TIMEOUT if a kernel gave up a wait.
+ */
+size_t int8_linear_forward_host_workspace_bytes(int64_t T, int64_t K, int64_t N);
+i8_status int8_linear_forward_host(const void* X_host, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                                   const void* bias, int64_t N, float threshold, void* Y_host,
+                                   int32_t* idx_host, int32_t* n_out_host, void* workspace,
+                                   size_t workspace_bytes, cudaStream_t stream);
+
+/* As int8_linear_forward_path, and records caller-created CUDA events
+ * (cudaEvent_t, passed as void*) on `stream` around the stages:
+ * events[0] before the first stage, events[1] after the outlier pass,
+ * events[2] after the row quantisation, events[3] after the product kernel.
+ * For measurement: event deltas time each kernel on its launching stream. */
+i8_status int8_linear_forward_timed(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                                    const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
+                                    int32_t* n_out, void* workspace, size_t workspace_bytes, int path,
+                                    void* const* events, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Inspection entry points (used by the parity tests; not needed for inference)
+ * ------------------------------------------------------------------------- */
+
+/* Byte offsets of the forward's intermediate buffers inside the workspace, so
+ * a caller can read the stage results of the most recent forward:
+ *   mask  uint32 [ceil(K/32)]  outlier column bitmask (bit k%32 of word k/32)
+ *   sA    fp32 [T]             row absmax over non-outlier columns
+ *   Xq    int8 [T,K]           row codes (outlier columns 0)
+ *   Xo    fp16 [T,ldo]         X[:, idx[o]] for o < n_out, zero up to a multiple of 64
+ *   Wo    fp16 [N,ldo]         fp16((CB[j,idx[o]]*SCB[j])/127), same padding
+ *                              (written by the tensor-core path only)
+ * ldo (elements) = K rounded up to a multiple of 64.  Host-only. */
+typedef struct int8_ws_layout {
+  uint64_t status, mask, sA, Xq, Xo, Wo, total;
+  int64_t ldo;
+} int8_ws_layout;
+i8_status int8_linear_workspace_layout(int64_t T, int64_t K, int64_t N, int8_ws_layout* out);
+
+/*
+ * Int8 product alone: acc[t,j] = sum_k Xq[t,k]*CB[j,k] (exact int32), with the
+ * same kernels as the forward (path 1 = tensor-core GEMM, path 2 = decode
+ * GEMV for T <= 16, 0 = automatic).
+ *   Xq device int8 [T,K], CB device int8 [N,K], acc device int32 [T,N].
+ *   workspace as for int8_linear_forward (only its status word is used).
+ */
+i8_status int8_gemm_i32(const int8_t* Xq, int64_t T, int64_t K, const int8_t* CB, int64_t N, int32_t* acc,
+                        int path, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The largest fp16 magnitude bit pattern (0..0x7bff) whose value is <= threshold;
+ * the outlier test |x| > threshold is (bits(x) & 0x7fff) > this value for
+ * non-NaN x.  Host-only; 0xffffffff when threshold <= 0 or NaN (no outliers). */
+uint32_t int8_outlier_threshold_bits(float threshold);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INT8MP_H_ */

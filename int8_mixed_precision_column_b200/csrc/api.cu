@@ -1,0 +1,319 @@
+// C ABI of libint8mp: argument validation, workspace layout and dispatch of
+// the LLM.int8() forward linear layer kernels.  See include/int8mp.h for the
+// contract of every entry point.
+#include <cmath>
+#include <cstring>
+
+#include "../../include/int8mp.h"
+#include "kernels.h"
+
+using namespace i8mp;
+
+namespace {
+
+constexpr int64_t kMaxK = 131072;      // K*127^2 < 2^31
+constexpr int64_t kMaxRows = int64_t(1) << 30;
+constexpr int kMaxDevices = 64;
+
+struct DevInfo {
+  bool probed = false;
+  bool sm100 = false;
+  int num_sms = 0;
+};
+DevInfo g_dev[kMaxDevices];
+
+i8_status device_info(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return I8_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return I8_ERR_UNSUPPORTED;
+  DevInfo& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return I8_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return I8_ERR_CUDA;
+    d.sm100 = (major == 10);
+    d.num_sms = sms;
+    d.probed = true;
+  }
+  if (!d.sm100) return I8_ERR_UNSUPPORTED;
+  *num_sms = d.num_sms;
+  return I8_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline uint64_t align_up(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
+
+bool shape_ok(int64_t T, int64_t K, int64_t N) {
+  return T >= 0 && T <= kMaxRows && K >= 16 && K % 16 == 0 && K <= kMaxK && N >= 16 && N % 16 == 0 &&
+         N <= kMaxRows;
+}
+
+int8_ws_layout make_layout(int64_t T, int64_t K, int64_t N) {
+  int8_ws_layout L;
+  L.ldo = ((K + 63) / 64) * 64;
+  L.status = 0;
+  L.mask = 256;
+  const uint64_t mask_bytes = static_cast<uint64_t>((K + 31) / 32) * 4;
+  L.sA = align_up(L.mask + mask_bytes, 256);
+  L.Xq = align_up(L.sA + static_cast<uint64_t>(T) * 4, 256);
+  L.Xo = align_up(L.Xq + static_cast<uint64_t>(T) * K, 256);
+  L.Wo = align_up(L.Xo + static_cast<uint64_t>(T) * L.ldo * 2, 256);
+  L.total = align_up(L.Wo + static_cast<uint64_t>(N) * L.ldo * 2, 256);
+  return L;
+}
+
+struct HostExtra {
+  uint64_t x, y, idx, n_out, total;
+};
+HostExtra make_host_extra(int64_t T, int64_t K, int64_t N) {
+  const int8_ws_layout L = make_layout(T, K, N);
+  HostExtra h;
+  h.x = L.total;
+  h.y = align_up(h.x + static_cast<uint64_t>(T) * K * 2, 256);
+  h.idx = align_up(h.y + static_cast<uint64_t>(T) * N * 2, 256);
+  h.n_out = align_up(h.idx + static_cast<uint64_t>(K) * 4, 256);
+  h.total = align_up(h.n_out + 4, 256);
+  return h;
+}
+
+float half_bits_value(uint32_t h) {
+  const uint32_t e = (h >> 10) & 0x1fu;
+  const uint32_t m = h & 0x3ffu;
+  if (e == 0) return std::ldexp(static_cast<float>(m), -24);
+  if (e == 31) return m == 0 ? INFINITY : NAN;
+  return std::ldexp(static_cast<float>(m | 0x400u), static_cast<int>(e) - 25);
+}
+
+uint32_t threshold_bits(float thr) {
+  if (!(thr > 0.0f)) return 0xffffffffu;
+  // largest pattern p in [0, 0x7c00] with value(p) <= thr; value is monotone in p.
+  uint32_t lo = 0, hi = 0x7c00;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi + 1) / 2;
+    if (half_bits_value(mid) <= thr)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+inline i8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? I8_OK : I8_ERR_CUDA; }
+
+i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB, const void* bias,
+                       int64_t N, float threshold, void* Y, int32_t* idx, int32_t* n_out, void* ws, size_t ws_bytes,
+                       int path, void* const* events, cudaStream_t stream) {
+  if (!shape_ok(T, K, N)) return I8_ERR_INVALID_ARG;
+  if (path < 0 || path > 2) return I8_ERR_INVALID_ARG;
+  if (path == 2 && T > kDecodeMaxT) return I8_ERR_INVALID_ARG;
+  if (idx == nullptr || n_out == nullptr || !aligned(idx, 4) || !aligned(n_out, 4)) return I8_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (X == nullptr || CB == nullptr || SCB == nullptr || Y == nullptr) return I8_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(CB, 16) || !aligned(Y, 16) || !aligned(SCB, 4) ||
+        (bias != nullptr && !aligned(bias, 2)))
+      return I8_ERR_INVALID_ARG;
+  }
+  const int8_ws_layout L = make_layout(T, K, N);
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < L.total) return I8_ERR_WORKSPACE;
+  int num_sms = 0;
+  i8_status st = device_info(&num_sms);
+  if (st != I8_OK) return st;
+
+  auto mark = [&](int i) -> bool {
+    return events == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) == cudaSuccess;
+  };
+  if (!mark(0)) return I8_ERR_CUDA;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const uint64_t mask_bytes = static_cast<uint64_t>((K + 31) / 32) * 4;
+  // status word + mask start at zero for every forward
+  cudaError_t e = cudaMemsetAsync(w, 0, L.mask + mask_bytes, stream);
+  if (e != cudaSuccess) return I8_ERR_CUDA;
+  if (T == 0) {
+    e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
+    return (e == cudaSuccess && mark(1) && mark(2) && mark(3)) ? I8_OK : I8_ERR_CUDA;
+  }
+
+  DevStatus* dst = reinterpret_cast<DevStatus*>(w + L.status);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(w + L.mask);
+  float* sA = reinterpret_cast<float*>(w + L.sA);
+  int8_t* Xq = reinterpret_cast<int8_t*>(w + L.Xq);
+  __half* Xo = reinterpret_cast<__half*>(w + L.Xo);
+  __half* Wo = reinterpret_cast<__half*>(w + L.Wo);
+  const __half* Xh = static_cast<const __half*>(X);
+
+  const uint32_t hb = threshold_bits(threshold);
+  if (hb == 0xffffffffu)
+    e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
+  else
+    e = launch_outliers(Xh, T, K, hb, mask, idx, n_out, dst, stream);
+  if (e != cudaSuccess || !mark(1)) return I8_ERR_CUDA;
+
+  const bool gemv = (path == 2) || (path == 0 && T <= kDecodeMaxT);
+  e = launch_rowquant(Xh, T, K, mask, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, stream);
+  if (e != cudaSuccess || !mark(2)) return I8_ERR_CUDA;
+
+  GemmArgs a;
+  a.Xq = Xq;
+  a.CB = CB;
+  a.Xo = Xo;
+  a.Wo = Wo;
+  a.ldo = L.ldo;
+  a.sA = sA;
+  a.SCB = SCB;
+  a.bias = static_cast<const __half*>(bias);
+  a.Y = static_cast<__half*>(Y);
+  a.acc_out = nullptr;
+  a.n_out = n_out;
+  a.idx = idx;
+  a.st = dst;
+  a.T = T;
+  a.N = N;
+  a.K = K;
+  a.mode = 0;
+  e = gemv ? launch_gemv_decode(a, num_sms, stream) : launch_gemm_tc(a, num_sms, stream);
+  if (e != cudaSuccess || !mark(3)) return I8_ERR_CUDA;
+  return I8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* int8_status_string(int status) {
+  switch (status) {
+    case I8_OK: return "I8_OK";
+    case I8_ERR_INVALID_ARG: return "I8_ERR_INVALID_ARG";
+    case I8_ERR_WORKSPACE: return "I8_ERR_WORKSPACE";
+    case I8_ERR_CUDA: return "I8_ERR_CUDA";
+    case I8_ERR_TIMEOUT: return "I8_ERR_TIMEOUT";
+    case I8_ERR_UNSUPPORTED: return "I8_ERR_UNSUPPORTED";
+    default: return "I8_ERR_UNKNOWN";
+  }
+}
+
+int int8_version(void) { return 100; }
+
+uint32_t int8_outlier_threshold_bits(float threshold) { return threshold_bits(threshold); }
+
+i8_status int8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* CB, float* SCB, cudaStream_t stream) {
+  if (N < 0 || N > kMaxRows || K < 16 || K % 16 != 0 || K > kMaxK) return I8_ERR_INVALID_ARG;
+  if (N == 0) return I8_OK;
+  if (W == nullptr || CB == nullptr || SCB == nullptr) return I8_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(CB, 8) || !aligned(SCB, 4)) return I8_ERR_INVALID_ARG;
+  int num_sms = 0;
+  i8_status st = device_info(&num_sms);
+  if (st != I8_OK) return st;
+  return cuda_status(launch_quantize_weight(static_cast<const __half*>(W), N, K, CB, SCB, stream));
+}
+
+size_t int8_linear_workspace_bytes(int64_t T, int64_t K, int64_t N) {
+  if (!shape_ok(T, K, N)) return 0;
+  return static_cast<size_t>(make_layout(T, K, N).total);
+}
+
+i8_status int8_linear_workspace_layout(int64_t T, int64_t K, int64_t N, int8_ws_layout* out) {
+  if (out == nullptr || !shape_ok(T, K, N)) return I8_ERR_INVALID_ARG;
+  *out = make_layout(T, K, N);
+  return I8_OK;
+}
+
+i8_status int8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                              const void* bias, int64_t N, float threshold, void* Y, int32_t* idx, int32_t* n_out,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return forward_impl(X, T, K, CB, SCB, bias, N, threshold, Y, idx, n_out, workspace, workspace_bytes, 0, nullptr,
+                      stream);
+}
+
+i8_status int8_linear_forward_path(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                                   const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
+                                   int32_t* n_out, void* workspace, size_t workspace_bytes, int path,
+                                   cudaStream_t stream) {
+  return forward_impl(X, T, K, CB, SCB, bias, N, threshold, Y, idx, n_out, workspace, workspace_bytes, path,
+                      nullptr, stream);
+}
+
+i8_status int8_linear_forward_timed(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                                    const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
+                                    int32_t* n_out, void* workspace, size_t workspace_bytes, int path,
+                                    void* const* events, cudaStream_t stream) {
+  if (events == nullptr) return I8_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i)
+    if (events[i] == nullptr) return I8_ERR_INVALID_ARG;
+  return forward_impl(X, T, K, CB, SCB, bias, N, threshold, Y, idx, n_out, workspace, workspace_bytes, path, events,
+                      stream);
+}
+
+i8_status int8_check_status(void* workspace, uint32_t* where, cudaStream_t stream) {
+  if (workspace == nullptr || !aligned(workspace, 256)) return I8_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return I8_ERR_CUDA;
+  DevStatus h;
+  if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return I8_ERR_CUDA;
+  if (where != nullptr) *where = h.where;
+  if (h.error == 0) return I8_OK;
+  if (cudaMemset(workspace, 0, 2 * sizeof(uint32_t)) != cudaSuccess) return I8_ERR_CUDA;
+  return h.error == kErrTimeout ? I8_ERR_TIMEOUT : I8_ERR_CUDA;
+}
+
+size_t int8_linear_forward_host_workspace_bytes(int64_t T, int64_t K, int64_t N) {
+  if (!shape_ok(T, K, N)) return 0;
+  return static_cast<size_t>(make_host_extra(T, K, N).total);
+}
+
+i8_status int8_linear_forward_host(const void* X_host, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                                   const void* bias, int64_t N, float threshold, void* Y_host, int32_t* idx_host,
+                                   int32_t* n_out_host, void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
+  if (!shape_ok(T, K, N)) return I8_ERR_INVALID_ARG;
+  if (T > 0 && (X_host == nullptr || Y_host == nullptr)) return I8_ERR_INVALID_ARG;
+  const HostExtra H = make_host_extra(T, K, N);
+  const int8_ws_layout L = make_layout(T, K, N);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < H.total) return I8_ERR_WORKSPACE;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  void* Xd = w + H.x;
+  void* Yd = w + H.y;
+  int32_t* idxd = reinterpret_cast<int32_t*>(w + H.idx);
+  int32_t* nd = reinterpret_cast<int32_t*>(w + H.n_out);
+  const size_t xbytes = static_cast<size_t>(T) * K * 2;
+  const size_t ybytes = static_cast<size_t>(T) * N * 2;
+  if (xbytes && cudaMemcpyAsync(Xd, X_host, xbytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return I8_ERR_CUDA;
+  i8_status st =
+      forward_impl(Xd, T, K, CB, SCB, bias, N, threshold, Yd, idxd, nd, workspace, L.total, 0, nullptr, stream);
+  if (st != I8_OK) return st;
+  if (ybytes && cudaMemcpyAsync(Y_host, Yd, ybytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return I8_ERR_CUDA;
+  if (idx_host && cudaMemcpyAsync(idx_host, idxd, static_cast<size_t>(K) * 4, cudaMemcpyDeviceToHost, stream) !=
+                      cudaSuccess)
+    return I8_ERR_CUDA;
+  if (n_out_host && cudaMemcpyAsync(n_out_host, nd, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return I8_ERR_CUDA;
+  return int8_check_status(workspace, nullptr, stream);
+}
+
+i8_status int8_gemm_i32(const int8_t* Xq, int64_t T, int64_t K, const int8_t* CB, int64_t N, int32_t* acc, int path,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!shape_ok(T, K, N) || path < 0 || path > 2) return I8_ERR_INVALID_ARG;
+  if (path == 2 && T > kDecodeMaxT) return I8_ERR_INVALID_ARG;
+  if (T > 0 && (Xq == nullptr || CB == nullptr || acc == nullptr)) return I8_ERR_INVALID_ARG;
+  if (T > 0 && (!aligned(Xq, 16) || !aligned(CB, 16) || !aligned(acc, 16))) return I8_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < sizeof(DevStatus)) return I8_ERR_WORKSPACE;
+  int num_sms = 0;
+  i8_status st = device_info(&num_sms);
+  if (st != I8_OK) return st;
+  if (cudaMemsetAsync(workspace, 0, sizeof(DevStatus), stream) != cudaSuccess) return I8_ERR_CUDA;
+  if (T == 0) return I8_OK;
+  GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.Xq = Xq;
+  a.CB = CB;
+  a.acc_out = acc;
+  a.st = static_cast<DevStatus*>(workspace);
+  a.T = T;
+  a.N = N;
+  a.K = K;
+  a.mode = 1;
+  const bool gemv = (path == 2) || (path == 0 && T <= kDecodeMaxT);
+  return cuda_status(gemv ? launch_gemv_decode(a, num_sms, stream) : launch_gemm_tc(a, num_sms, stream));
+}
+
+}  // extern "C"

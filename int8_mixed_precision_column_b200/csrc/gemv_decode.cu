@@ -1,0 +1,170 @@
+// Decode-regime (1..16 tokens) int8 product of the LLM.int8() forward linear
+// layer: the same decomposition as the prefill GEMM (int8 vector-wise product
+// over the non-outlier columns, 16-bit product over the outlier columns,
+// dequantise and sum; "Core idea of LLM.int8()", Hugging Face integration
+// page), shaped for streaming the int8 weight CB from HBM once.
+//
+// Work split: output rows are taken in groups of 8; each CTA owns a contiguous,
+// balanced range of groups and walks it 4 groups (32 rows) at a time.  The 8
+// warps of a CTA split K; each warp multiplies its K-slice of the 16 x K token
+// codes by the 32 weight rows with mma.sync m16n8k32 (s8 x s8 -> s32), and the
+// warps' int32 partial sums are added in shared memory (exact).
+// Fragment trick: the dot product is a sum over k, so any permutation of k
+// applied to both operands leaves it unchanged.  Thread (g, t) of a warp loads
+// 16 contiguous bytes of weight row g at k0 + 16t and the same 16 bytes of
+// token rows g and g+8; two MMAs consume them (bytes 0-7, then 8-15).
+// Epilogue: Y = fp16(acc * sA[t] * SCB[j] / 127^2 + sum_o Xo[t,o] * Wo[j,o] + b[j])
+// with Wo[j,o] = fp16((CB[j, idx[o]] * SCB[j]) / 127) recomputed from CB.
+#include "kernels.h"
+
+namespace i8mp {
+namespace {
+
+constexpr int DV_WARPS = 8;
+constexpr int DV_THREADS = DV_WARPS * 32;
+constexpr int DV_RG = 4;  // 8-row groups per pass
+
+struct DvParams {
+  const int8_t* Xq;
+  const float* sA;
+  const int8_t* CB;
+  const float* SCB;
+  const __half* bias;
+  const __half* Xo;
+  int64_t ldo;
+  const int32_t* idx;
+  const int32_t* n_out;
+  __half* Y;
+  int32_t* acc_out;
+  int64_t T, N, K;
+  int mode;
+};
+
+__device__ __forceinline__ void mma_s8_16832(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ld_stream(const int8_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__global__ void __launch_bounds__(DV_THREADS) gemv_i8_decode_kernel(const DvParams p) {
+  __shared__ int32_t red[DV_WARPS][DV_RG][32][4];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int t4 = lane & 3;
+  const int64_t G = p.N / 8;
+  const int64_t g_begin = G * blockIdx.x / gridDim.x;
+  const int64_t g_end = G * (blockIdx.x + 1) / gridDim.x;
+  const int64_t steps = (p.K + 63) / 64;
+  const int64_t s_begin = steps * warp / DV_WARPS;
+  const int64_t s_end = steps * (warp + 1) / DV_WARPS;
+  const int n_out = (p.mode == 0) ? *p.n_out : 0;
+  const bool row_a = g < p.T;
+  const bool row_b = g + 8 < p.T;
+  const int8_t* xa_base = p.Xq + static_cast<int64_t>(g) * p.K + t4 * 16;
+  const int8_t* xb_base = p.Xq + static_cast<int64_t>(g + 8) * p.K + t4 * 16;
+
+  for (int64_t g0 = g_begin; g0 < g_end; g0 += DV_RG) {
+    int32_t c[DV_RG][4];
+    #pragma unroll
+    for (int r = 0; r < DV_RG; ++r) c[r][0] = c[r][1] = c[r][2] = c[r][3] = 0;
+    const int8_t* wrow[DV_RG];
+    bool wok[DV_RG];
+    #pragma unroll
+    for (int r = 0; r < DV_RG; ++r) {
+      wok[r] = (g0 + r) < g_end;
+      wrow[r] = p.CB + ((g0 + r) * 8 + g) * p.K + t4 * 16;
+    }
+    #pragma unroll 2
+    for (int64_t st = s_begin; st < s_end; ++st) {
+      const int64_t k = st * 64;
+      const bool kok = k + t4 * 16 < p.K;
+      uint4 w[DV_RG];
+      #pragma unroll
+      for (int r = 0; r < DV_RG; ++r) w[r] = (wok[r] && kok) ? ld_stream(wrow[r] + k) : make_uint4(0, 0, 0, 0);
+      const uint4 xa = (row_a && kok) ? __ldg(reinterpret_cast<const uint4*>(xa_base + k)) : make_uint4(0, 0, 0, 0);
+      const uint4 xb = (row_b && kok) ? __ldg(reinterpret_cast<const uint4*>(xb_base + k)) : make_uint4(0, 0, 0, 0);
+      #pragma unroll
+      for (int r = 0; r < DV_RG; ++r) {
+        mma_s8_16832(c[r], xa.x, xb.x, xa.y, xb.y, w[r].x, w[r].y);
+        mma_s8_16832(c[r], xa.z, xb.z, xa.w, xb.w, w[r].z, w[r].w);
+      }
+    }
+    #pragma unroll
+    for (int r = 0; r < DV_RG; ++r) {
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) red[warp][r][lane][i] = c[r][i];
+    }
+    __syncthreads();
+    // 4 groups x 32 lanes x 4 values = 512 outputs (token, row) per pass.
+    for (int v = threadIdx.x; v < DV_RG * 128; v += DV_THREADS) {
+      const int r = v >> 7;
+      const int ln = (v >> 2) & 31;
+      const int i = v & 3;
+      if (g0 + r >= g_end) continue;
+      const int tok = (ln >> 2) + ((i >> 1) << 3);
+      if (tok >= p.T) continue;
+      const int64_t j = (g0 + r) * 8 + (ln & 3) * 2 + (i & 1);
+      int32_t acc = 0;
+      #pragma unroll
+      for (int w = 0; w < DV_WARPS; ++w) acc += red[w][r][ln][i];
+      if (p.mode == 1) {
+        p.acc_out[tok * p.N + j] = acc;
+        continue;
+      }
+      const float scb = __ldg(&p.SCB[j]);
+      float y = static_cast<float>(acc) * (__ldg(&p.sA[tok]) * (1.0f / 16129.0f) * scb);
+      float yo = 0.0f;
+      for (int o = 0; o < n_out; ++o) {
+        const float cbv = static_cast<float>(__ldg(&p.CB[j * p.K + __ldg(&p.idx[o])]));
+        const float wo = __half2float(__float2half_rn(__fdiv_rn(__fmul_rn(cbv, scb), 127.0f)));
+        yo = fmaf(__half2float(p.Xo[tok * p.ldo + o]), wo, yo);
+      }
+      y += yo;
+      if (p.bias != nullptr) y += __half2float(p.bias[j]);
+      p.Y[tok * p.N + j] = __float2half_rn(y);
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s) {
+  if (a.T == 0 || a.N == 0) return cudaSuccess;
+  if (a.T > kDecodeMaxT) return cudaErrorInvalidValue;
+  DvParams p;
+  p.Xq = a.Xq;
+  p.sA = a.sA;
+  p.CB = a.CB;
+  p.SCB = a.SCB;
+  p.bias = a.bias;
+  p.Xo = a.Xo;
+  p.ldo = a.ldo;
+  p.idx = a.idx;
+  p.n_out = a.n_out;
+  p.Y = a.Y;
+  p.acc_out = a.acc_out;
+  p.T = a.T;
+  p.N = a.N;
+  p.K = a.K;
+  p.mode = a.mode;
+  const int64_t groups = a.N / 8;
+  int64_t grid = static_cast<int64_t>(num_sms) * 2;
+  if (grid > groups) grid = groups;
+  gemv_i8_decode_kernel<<<static_cast<unsigned>(grid), DV_THREADS, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace i8mp

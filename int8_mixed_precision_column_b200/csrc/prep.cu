@@ -1,0 +1,300 @@
+// Memory-bound stages of the LLM.int8() forward linear layer:
+//  * weight absmax quantisation (CB int8, SCB fp32), done once per layer;
+//  * the column outlier mask and its compaction into the ascending index list;
+//  * row-wise absmax int8 quantisation of the non-outlier activations, and the
+//    gathers that feed the 16-bit outlier product.
+//
+// Method: "Hugging Face integrates LLM.int8() 8-bit matrix multiplication into
+// Transformers and Accelerate", sections "Core idea of LLM.int8()" (steps 1-2)
+// and "Quantization mechanics" (absmax, 127/absmax, codes in [-127, 127]);
+// bitsandbytes Linear8bitLt docstring (threshold acts on activation columns);
+// bitsandbytes issue #1609 (state.idx lists the outlier columns).
+#include "kernels.h"
+
+namespace i8mp {
+
+// ---------------------------------------------------------------------------
+// Weight quantisation: one warp per output row j.
+// SCB[j] = max_k |W[j,k]|; CB[j,k] = clamp(roundf(W[j,k] * (127/SCB[j])), +-127).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quantize_weight_kernel(const __half* __restrict__ W, int64_t N, int64_t K,
+                                                              int8_t* __restrict__ CB, float* __restrict__ SCB) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const int64_t nv = K / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(W + row * K);
+  float m = 0.0f;
+  for (int64_t i = lane; i < nv; i += 32) {
+    uint4 v = __ldg(src + i);
+    const __half* h = reinterpret_cast<const __half*>(&v);
+    #pragma unroll
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(__half2float(h[e])));
+  }
+  m = warp_max(m);
+  const float inv = scale_inv(m);
+  if (lane == 0) SCB[row] = m;
+  uint2* dst = reinterpret_cast<uint2*>(CB + row * K);
+  for (int64_t i = lane; i < nv; i += 32) {
+    uint4 v = __ldg(src + i);
+    const __half* h = reinterpret_cast<const __half*>(&v);
+    uint32_t lo = 0, hi = 0;
+    #pragma unroll
+    for (int e = 0; e < 4; ++e) lo |= (static_cast<uint32_t>(quant_code(__half2float(h[e]), inv)) & 0xffu) << (8 * e);
+    #pragma unroll
+    for (int e = 0; e < 4; ++e) hi |= (static_cast<uint32_t>(quant_code(__half2float(h[4 + e]), inv)) & 0xffu) << (8 * e);
+    dst[i] = make_uint2(lo, hi);
+  }
+}
+
+cudaError_t launch_quantize_weight(const __half* W, int64_t N, int64_t K, int8_t* CB, float* SCB, cudaStream_t s) {
+  if (N == 0) return cudaSuccess;
+  const int64_t blocks = (N + 7) / 8;
+  quantize_weight_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(W, N, K, CB, SCB);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Column outlier mask.
+//
+// Grid: x = 256-column slabs, y = row chunks.  Each thread owns 8 consecutive
+// columns (one 16-byte load per row) and ORs together, over its rows, the bits
+// "|x| > threshold".  The comparison is done on fp16 magnitude bit patterns:
+// for non-NaN fp16 values the magnitude order equals the order of the 15-bit
+// patterns, so |x| > threshold  <=>  (bits & 0x7fff) > hbits, where hbits is
+// the largest pattern whose value is <= threshold (computed on the host).
+// NaN patterns (> 0x7c00) are excluded so that NaN never flags a column.
+// The CTA merges its 8 warps in shared memory and ORs 8 words into the mask.
+// The last CTA to finish compacts the mask into the ascending idx list.
+// ---------------------------------------------------------------------------
+constexpr int kMaskThreads = 256;
+constexpr int kMaskRowsPerChunk = 128;
+
+__device__ __forceinline__ uint32_t flag_bits8(const uint4& v, uint32_t h2) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t bits = 0;
+  #pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t a = w[i] & 0x7fff7fffu;
+    const uint32_t m = __vcmpgtu2(a, h2) & __vcmpleu2(a, 0x7c007c00u);
+    bits |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * i);
+  }
+  return bits;
+}
+
+__global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const __half* __restrict__ X, int64_t T, int64_t K,
+                                                                    uint32_t hbits, uint32_t* __restrict__ mask,
+                                                                    int32_t* __restrict__ idx, int32_t* __restrict__ n_out,
+                                                                    DevStatus* st) {
+  __shared__ uint32_t s_words[8];
+  __shared__ int s_last;
+  __shared__ int s_scan[kMaskThreads];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int64_t col8 = static_cast<int64_t>(blockIdx.x) * 256 + lane * 8;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kMaskRowsPerChunk;
+  const int64_t r1 = min(T, r0 + kMaskRowsPerChunk);
+  const uint32_t h2 = hbits | (hbits << 16);
+  if (threadIdx.x < 8) s_words[threadIdx.x] = 0;
+  __syncthreads();
+
+  uint32_t bits = 0;
+  if (col8 < K) {
+    const __half* base = X + col8;
+    int64_t r = r0 + warp;
+    #pragma unroll 1
+    for (; r + 24 < r1; r += 32) {
+      uint4 v0 = __ldg(reinterpret_cast<const uint4*>(base + (r + 0) * K));
+      uint4 v1 = __ldg(reinterpret_cast<const uint4*>(base + (r + 8) * K));
+      uint4 v2 = __ldg(reinterpret_cast<const uint4*>(base + (r + 16) * K));
+      uint4 v3 = __ldg(reinterpret_cast<const uint4*>(base + (r + 24) * K));
+      bits |= flag_bits8(v0, h2) | flag_bits8(v1, h2) | flag_bits8(v2, h2) | flag_bits8(v3, h2);
+    }
+    #pragma unroll 1
+    for (; r < r1; r += 8) bits |= flag_bits8(__ldg(reinterpret_cast<const uint4*>(base + r * K)), h2);
+  }
+  if (bits) atomicOr(&s_words[lane >> 2], bits << ((lane & 3) * 8));
+  __syncthreads();
+  const int64_t nwords = (K + 31) / 32;
+  if (threadIdx.x < 8) {
+    const int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + threadIdx.x;
+    if (w < nwords && s_words[threadIdx.x]) atomicOr(&mask[w], s_words[threadIdx.x]);
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t total = gridDim.x * gridDim.y;
+    const uint32_t prev = atomicAdd(&st->counter, 1u);
+    s_last = (prev == total - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  // Compaction: thread t owns a contiguous run of mask words, so a block-wide
+  // exclusive scan of per-thread popcounts yields ascending positions.
+  const int64_t per = (nwords + kMaskThreads - 1) / kMaskThreads;
+  const int64_t w0 = threadIdx.x * per;
+  const int64_t w1 = min(nwords, w0 + per);
+  int cnt = 0;
+  for (int64_t w = w0; w < w1; ++w) cnt += __popc(__ldcg(&mask[w]));
+  s_scan[threadIdx.x] = cnt;
+  __syncthreads();
+  for (int off = 1; off < kMaskThreads; off <<= 1) {
+    int v = (threadIdx.x >= off) ? s_scan[threadIdx.x - off] : 0;
+    __syncthreads();
+    s_scan[threadIdx.x] += v;
+    __syncthreads();
+  }
+  int pos = s_scan[threadIdx.x] - cnt;
+  for (int64_t w = w0; w < w1; ++w) {
+    uint32_t m = __ldcg(&mask[w]);
+    while (m) {
+      const int b = __ffs(m) - 1;
+      m &= m - 1;
+      idx[pos++] = static_cast<int32_t>(w * 32 + b);
+    }
+  }
+  if (threadIdx.x == kMaskThreads - 1) {
+    *n_out = s_scan[kMaskThreads - 1];
+    st->counter = 0;
+  }
+}
+
+cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask, int32_t* idx,
+                            int32_t* n_out, DevStatus* st, cudaStream_t s) {
+  const int64_t slabs = (K + 255) / 256;
+  const int64_t chunks = (T + kMaskRowsPerChunk - 1) / kMaskRowsPerChunk;
+  if (slabs > 0x7fffffff || chunks > 65535) return cudaErrorInvalidValue;
+  dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(chunks));
+  outlier_mask_kernel<<<grid, kMaskThreads, 0, s>>>(X, T, K, hbits, mask, idx, n_out, st);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Row quantisation + outlier gathers.
+//
+// Blocks [0, T): one CTA per token row t.  The row is read once into registers
+// (8 columns per 16-byte chunk), the absmax over non-outlier columns is
+// reduced across the CTA, and the codes are written as 8-byte packets.  The
+// CTA then writes the row of Xo: X[t, idx[o]] for o < n_out, zero up to the
+// next multiple of 64 (the K-block of the fp16 outlier MMA).
+// Blocks [T, T + ceil(N/kWoRows)): rows of Wo = fp16((CB[j, idx[o]] * SCB[j]) / 127),
+// zero-padded the same way (only when the tensor-core path consumes Wo).
+// ---------------------------------------------------------------------------
+constexpr int kRowThreads = 256;
+constexpr int kRowChunks = 8;   // registers hold rows up to 256*8*8 = 16384 columns
+constexpr int kWoRows = 32;
+
+__device__ __forceinline__ uint32_t mask_byte(const uint32_t* mask, int64_t chunk) {
+  return (__ldg(&mask[chunk >> 2]) >> ((chunk & 3) * 8)) & 0xffu;
+}
+
+__device__ __forceinline__ float row_absmax_part(const uint4& v, uint32_t mb) {
+  const __half* h = reinterpret_cast<const __half*>(&v);
+  float m = 0.0f;
+  #pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if (!((mb >> e) & 1u)) m = fmaxf(m, fabsf(__half2float(h[e])));
+  return m;
+}
+
+__device__ __forceinline__ uint2 row_codes(const uint4& v, uint32_t mb, float inv) {
+  const __half* h = reinterpret_cast<const __half*>(&v);
+  uint32_t w[2] = {0u, 0u};
+  #pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int q = ((mb >> e) & 1u) ? 0 : quant_code(__half2float(h[e]), inv);
+    w[e >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (e & 3));
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+__global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
+    const __half* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p, int8_t* __restrict__ Xq,
+    float* __restrict__ sA, __half* __restrict__ Xo, int64_t ldo, const int8_t* __restrict__ CB,
+    const float* __restrict__ SCB, int64_t N, __half* __restrict__ Wo, int with_wo) {
+  __shared__ float s_red[kRowThreads / 32];
+  const int tid = threadIdx.x;
+  const int n_out = *n_out_p;
+  const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
+
+  if (static_cast<int64_t>(blockIdx.x) >= T) {
+    // ---- Wo rows ----
+    if (!with_wo || n_out == 0) return;
+    const int64_t j0 = (static_cast<int64_t>(blockIdx.x) - T) * kWoRows;
+    const int64_t total = static_cast<int64_t>(kWoRows) * npad;
+    for (int64_t e = tid; e < total; e += kRowThreads) {
+      const int64_t j = j0 + e / npad;
+      const int64_t o = e % npad;
+      if (j >= N) break;
+      __half v = __float2half_rn(0.0f);
+      if (o < n_out) {
+        const float c = static_cast<float>(__ldg(&CB[j * K + __ldg(&idx[o])]));
+        v = __float2half_rn(__fdiv_rn(__fmul_rn(c, __ldg(&SCB[j])), 127.0f));
+      }
+      Wo[j * ldo + o] = v;
+    }
+    return;
+  }
+
+  // ---- one token row ----
+  const int64_t t = blockIdx.x;
+  const int64_t nv = K / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(X + t * K);
+  uint4 v[kRowChunks];
+  uint32_t mb[kRowChunks];
+  float m = 0.0f;
+  #pragma unroll
+  for (int c = 0; c < kRowChunks; ++c) {
+    const int64_t i = tid + static_cast<int64_t>(c) * kRowThreads;
+    if (i < nv) {
+      v[c] = __ldcs(src + i);
+      mb[c] = mask_byte(mask, i);
+      m = fmaxf(m, row_absmax_part(v[c], mb[c]));
+    }
+  }
+  for (int64_t i = tid + static_cast<int64_t>(kRowChunks) * kRowThreads; i < nv; i += kRowThreads)
+    m = fmaxf(m, row_absmax_part(__ldg(src + i), mask_byte(mask, i)));
+  m = warp_max(m);
+  if ((tid & 31) == 0) s_red[tid >> 5] = m;
+  __syncthreads();
+  if (tid < 32) {
+    float r = (tid < kRowThreads / 32) ? s_red[tid] : 0.0f;
+    r = warp_max(r);
+    if (tid == 0) s_red[0] = r;
+  }
+  __syncthreads();
+  const float absmax = s_red[0];
+  const float inv = scale_inv(absmax);
+  if (tid == 0) sA[t] = absmax;
+  uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
+  #pragma unroll
+  for (int c = 0; c < kRowChunks; ++c) {
+    const int64_t i = tid + static_cast<int64_t>(c) * kRowThreads;
+    if (i < nv) dst[i] = row_codes(v[c], mb[c], inv);
+  }
+  for (int64_t i = tid + static_cast<int64_t>(kRowChunks) * kRowThreads; i < nv; i += kRowThreads)
+    dst[i] = row_codes(__ldg(src + i), mask_byte(mask, i), inv);
+
+  if (n_out > 0) {
+    const __half* xrow = X + t * K;
+    for (int64_t o = tid; o < npad; o += kRowThreads)
+      Xo[t * ldo + o] = (o < n_out) ? xrow[__ldg(&idx[o])] : __float2half_rn(0.0f);
+  }
+}
+
+cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_t* mask, const int32_t* idx,
+                            const int32_t* n_out, int8_t* Xq, float* sA, __half* Xo, int64_t ldo, const int8_t* CB,
+                            const float* SCB, int64_t N, __half* Wo, bool with_wo, cudaStream_t s) {
+  const int64_t wo_blocks = with_wo ? (N + kWoRows - 1) / kWoRows : 0;
+  const int64_t blocks = T + wo_blocks;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  rowquant_kernel<<<static_cast<unsigned>(blocks), kRowThreads, 0, s>>>(X, T, K, mask, idx, n_out, Xq, sA, Xo, ldo,
+                                                                        CB, SCB, N, Wo, with_wo ? 1 : 0);
+  return cudaGetLastError();
+}
+
+}  // namespace i8mp
