@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(m_blk) * BM + q * 32 + lane;
       const bool row_ok = row < p.T;
-      const float ra = row_ok ? __ldg(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
+      const float ra = (row_ok && p.mode == 0) ? __ldg(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
       #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         const int col0 = half * 128 + c * 32;
