@@ -183,6 +183,41 @@ i8_status int8_gemm_i32(const int8_t* Xq, int64_t T, int64_t K, const int8_t* CB
  * non-NaN x.  Host-only; 0xffffffff when threshold <= 0 or NaN (no outliers). */
 uint32_t int8_outlier_threshold_bits(float threshold);
 
+/* ---------------------------------------------------------------------------
+ * Forward without any caller-provided or allocated scratch memory.
+ *
+ * The pages have no counterpart to this call: it exists for callers that
+ * cannot allocate device memory and cannot pass a workspace -- for example a
+ * plugin inside an inference runtime that owns all device memory and forbids
+ * allocation during its execute call (cudaMalloc may synchronise the device
+ * and escapes the host's memory accounting), or an application with a fixed
+ * device-memory budget.
+ *
+ * Same arguments and results as int8_linear_forward for the decode case
+ * (1 <= T <= 16, same kernels, same integer stages), minus the workspace:
+ * the intermediate buffers live in a 4 MiB array compiled into the library
+ * (a file-scope __device__ array, held by every GPU that loads the library
+ * until the process exits).  It allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library call).
+ *   - Size limit: the scratch holds 256 B + 4*ceil(K/32) + 4*T + T*K +
+ *     2*T*ceil(K/64)*64 bytes (each part rounded up to 256 B); a T x K that
+ *     needs more than 4 MiB (for T = 16: K above about 87000) is rejected
+ *     with I8_ERR_WORKSPACE before any work is enqueued.  T outside
+ *     [1, 16] is I8_ERR_INVALID_ARG.
+ *   - The first call on each device resolves the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array, and the array keeps the
+ *     previous call's contents (each call clears what must start at zero).
+ *     Calls that can overlap on the GPU (other streams, other host threads)
+ *     race on it: serialise them.
+ *   - These kernels contain no device-side waits, so there is no status word
+ *     to read back.
+ */
+i8_status int8_linear_forward_decode_static(const void* X, int64_t T, int64_t K, const int8_t* CB,
+                                            const float* SCB, const void* bias, int64_t N, float threshold,
+                                            void* Y, int32_t* idx, int32_t* n_out, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
