@@ -178,6 +178,15 @@ i8_status int8_linear_workspace_layout(int64_t T, int64_t K, int64_t N, int8_ws_
 i8_status int8_gemm_i32(const int8_t* Xq, int64_t T, int64_t K, const int8_t* CB, int64_t N, int32_t* acc,
                         int path, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Self-test of failure detection: launches one thread that waits, with a
+ * limit of `limit_us` microseconds (1 .. 2000000), on an mbarrier that nothing
+ * arrives on -- the same bounded wait the tensor-core GEMM uses for every
+ * pipeline barrier.  The wait gives up, records I8_ERR_TIMEOUT (tag 0x5e1f) in
+ * the workspace status word and returns; int8_check_status() then reports it,
+ * and the CUDA context stays usable.  Nothing faults, traps or hangs. */
+i8_status int8_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t limit_us,
+                                     cudaStream_t stream);
+
 /* The largest fp16 magnitude bit pattern (0..0x7bff) whose value is <= threshold;
  * the outlier test |x| > threshold is (bits(x) & 0x7fff) > this value for
  * non-NaN x.  Host-only; 0xffffffff when threshold <= 0 or NaN (no outliers). */

@@ -77,11 +77,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 
 // Wait until the phase with the given parity has completed.  Gives up after
-// kWaitLimitNs (reporting kErrTimeout with tag `where` and raising *abort), or
+// limit_ns (default kWaitLimitNs; reporting kErrTimeout with tag `where` and raising *abort), or
 // as soon as another role of the CTA has raised *abort.  Returns false when it
 // gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          DevStatus* st, uint32_t where) {
+                                          DevStatus* st, uint32_t where, uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   #pragma unroll 1
   for (int i = 0; i < 256; ++i)
@@ -91,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   while (true) {
     if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1;
       report_error(st, kErrTimeout, where);
       return false;

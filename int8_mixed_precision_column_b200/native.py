@@ -58,6 +58,7 @@ SIGNATURES = {
     "int8_linear_workspace_layout": (_I32, [_I64, _I64, _I64, ctypes.POINTER(WsLayout)]),
     "int8_gemm_i32": (_I32, [_P, _I64, _I64, _P, _I64, _P, _I32, _P, _SZ, _P]),
     "int8_outlier_threshold_bits": (ctypes.c_uint32, [_F32]),
+    "int8_selftest_wait_timeout": (_I32, [_P, _SZ, ctypes.c_uint32, _P]),
     "int8_linear_forward_decode_static": (_I32, [_P, _I64, _I64, _P, _P, _P, _I64, _F32, _P, _P, _P, _P]),
 }
 
