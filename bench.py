@@ -190,6 +190,8 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     build.build()
     native.lib()
     p = WORKLOADS[args.workload]("cuda", rank_seed(rank))
+    if args.threshold is not None:
+        p.threshold = args.threshold
     T, K, N = p.T, p.K, p.N
     bias = p.bias
     CB, SCB = native.int8_quantize_weight(p.W)
@@ -213,7 +215,7 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
 
     def step(i):
-        native.int8_linear_forward_timed(X, CB, SCB, bias, p.threshold, Y, idx, n_out, ws, ev[i])
+        native.int8_linear_forward_timed(X, CB, SCB, bias, p.threshold, Y, idx, n_out, ws, ev[i], path=args.path)
 
     for i in range(args.warmup):
         if flush:
@@ -287,7 +289,7 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     work = algorithmic_work(T, K, N, n_outliers)
     peaks, peak_src = load_peaks()
     prod_avg = statistics.mean(prod_ms)
-    decode = T <= 16
+    decode = T <= 16 if args.path == 0 else args.path == 2
     if decode:
         achieved = work["product_bytes"] / (prod_avg * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -298,7 +300,8 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
         peak = peaks["bf16_tflops"] * INT8_PER_BF16
         achieved = work["int8_ops"] / (prod_avg * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS",
-                "frac": achieved / peak, "traffic": None, "kernel": "gemm_i8_tc_kernel",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "gemm_i8_tc_kernel" if args.path == 3 else "gemm_i8_tc2_kernel",
                 "peak_source": f"{peak_src} bf16_tflops (burst) x {INT8_PER_BF16} nominal int8:bf16 ratio",
                 "algorithmic_ops_per_launch": work["int8_ops"], "ms_per_launch": prod_avg}
     launches_per_step = 3 if p.threshold > 0 else 2
@@ -317,7 +320,7 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
         "vs_baseline": None,
         "dtype": "int8 x int8 -> int32 (+ fp16 outlier product, fp32 accumulate), fp16 in/out",
         "data": "synthetic (seeded; X ~ N(0,1) with planted outlier columns, W ~ N(0, 0.02^2))",
-        "config": {"workload": args.workload, "T": T, "K": K, "N": N, "threshold": p.threshold,
+        "config": {"workload": args.workload, "T": T, "K": K, "N": N, "threshold": p.threshold, "path": args.path,
                    "n_out": n_outliers, "parallelism": f"independent problem per rank x{world}",
                    "l2": "L2 flushed between steps" if flush else "inputs larger than L2 (no flush)"},
         "stage_ms": {"outliers": statistics.mean(outl_ms), "rowquant": statistics.mean(rowq_ms),
@@ -424,6 +427,10 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--threshold", type=float, default=None,
+                    help="override the workload's outlier threshold (<= 0 switches the decomposition off)")
+    ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="product kernel: 0 auto, 1 tensor core (SM pairs), 2 decode GEMV, 3 tensor core (single SM)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

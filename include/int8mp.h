@@ -108,8 +108,10 @@ i8_status int8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t*
                               cudaStream_t stream);
 
 /* As int8_linear_forward, with the product kernel chosen explicitly:
- * path 0 = automatic (as above), 1 = tensor-core GEMM (any T),
- * 2 = decode GEMV (T <= 16, else I8_ERR_INVALID_ARG). */
+ * path 0 = automatic (as above), 1 = tensor-core GEMM (any T; SM pairs with
+ * 256x256 tiles when 2-CTA clusters can be launched), 2 = decode GEMV
+ * (T <= 16, else I8_ERR_INVALID_ARG), 3 = tensor-core GEMM on single SMs
+ * (128x256 tiles). */
 i8_status int8_linear_forward_path(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
                                    const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
                                    int32_t* n_out, void* workspace, size_t workspace_bytes, int path,
@@ -155,7 +157,9 @@ i8_status int8_linear_forward_timed(const void* X, int64_t T, int64_t K, const i
 
 /* Byte offsets of the forward's intermediate buffers inside the workspace, so
  * a caller can read the stage results of the most recent forward:
- *   mask  uint32 [ceil(K/32)]  outlier column bitmask (bit k%32 of word k/32)
+ *   mask  uint32 [ceil(K/32)]  outlier column bitmask (bit k%32 of word k/32),
+ *                              followed by uint32 [ceil(K/32)] prefix counts
+ *                              (outlier columns in the words before each word)
  *   sA    fp32 [T]             row absmax over non-outlier columns
  *   Xq    int8 [T,K]           row codes (outlier columns 0)
  *   Xo    fp16 [T,ldo]         X[:, idx[o]] for o < n_out, zero up to a multiple of 64
@@ -170,8 +174,8 @@ i8_status int8_linear_workspace_layout(int64_t T, int64_t K, int64_t N, int8_ws_
 
 /*
  * Int8 product alone: acc[t,j] = sum_k Xq[t,k]*CB[j,k] (exact int32), with the
- * same kernels as the forward (path 1 = tensor-core GEMM, path 2 = decode
- * GEMV for T <= 16, 0 = automatic).
+ * same kernels as the forward (path 1 = tensor-core GEMM on SM pairs, 2 =
+ * decode GEMV for T <= 16, 3 = tensor-core GEMM on single SMs, 0 = automatic).
  *   Xq device int8 [T,K], CB device int8 [N,K], acc device int32 [T,N].
  *   workspace as for int8_linear_forward (only its status word is used).
  */
@@ -208,7 +212,7 @@ uint32_t int8_outlier_threshold_bits(float threshold);
  * (a file-scope __device__ array, held by every GPU that loads the library
  * until the process exits).  It allocates nothing (no cudaMalloc, cudaFree or
  * allocating library call).
- *   - Size limit: the scratch holds 256 B + 4*ceil(K/32) + 4*T + T*K +
+ *   - Size limit: the scratch holds 256 B + 8*ceil(K/32) + 4*T + T*K +
  *     2*T*ceil(K/64)*64 bytes (each part rounded up to 256 B); a T x K that
  *     needs more than 4 MiB (for T = 16: K above about 87000) is rejected
  *     with I8_ERR_WORKSPACE before any work is enqueued.  T outside

@@ -4,7 +4,7 @@
 #include <cmath>
 #include <cstring>
 
-#include "../../include/int8mp.h"
+#include "int8mp.h"
 #include "kernels.h"
 
 using namespace i8mp;
@@ -53,8 +53,9 @@ int8_ws_layout make_layout(int64_t T, int64_t K, int64_t N) {
   L.ldo = ((K + 63) / 64) * 64;
   L.status = 0;
   L.mask = 256;
+  // mask words, then the per-word prefix counts of the outlier columns
   const uint64_t mask_bytes = static_cast<uint64_t>((K + 31) / 32) * 4;
-  L.sA = align_up(L.mask + mask_bytes, 256);
+  L.sA = align_up(L.mask + 2 * mask_bytes, 256);
   L.Xq = align_up(L.sA + static_cast<uint64_t>(T) * 4, 256);
   L.Xo = align_up(L.Xq + static_cast<uint64_t>(T) * K, 256);
   L.Wo = align_up(L.Xo + static_cast<uint64_t>(T) * L.ldo * 2, 256);
@@ -100,12 +101,20 @@ uint32_t threshold_bits(float thr) {
 
 inline i8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? I8_OK : I8_ERR_CUDA; }
 
+// The product kernel: decode GEMV, or the tensor-core GEMM on SM pairs (the
+// single-SM GEMM when pairs are not launchable or when asked for explicitly).
+cudaError_t launch_product(const GemmArgs& a, int path, bool gemv, int num_sms, cudaStream_t stream) {
+  if (gemv) return launch_gemv_decode(a, num_sms, stream);
+  if (path != kPathTensorCoreSingleSM && pair_kernel_max_clusters() > 0) return launch_gemm_tc2(a, stream);
+  return launch_gemm_tc(a, num_sms, stream);
+}
+
 i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB, const void* bias,
                        int64_t N, float threshold, void* Y, int32_t* idx, int32_t* n_out, void* ws, size_t ws_bytes,
                        int path, void* const* events, cudaStream_t stream) {
   if (!shape_ok(T, K, N)) return I8_ERR_INVALID_ARG;
-  if (path < 0 || path > 2) return I8_ERR_INVALID_ARG;
-  if (path == 2 && T > kDecodeMaxT) return I8_ERR_INVALID_ARG;
+  if (path < kPathAuto || path > kPathTensorCoreSingleSM) return I8_ERR_INVALID_ARG;
+  if (path == kPathDecode && T > kDecodeMaxT) return I8_ERR_INVALID_ARG;
   if (idx == nullptr || n_out == nullptr || !aligned(idx, 4) || !aligned(n_out, 4)) return I8_ERR_INVALID_ARG;
   if (T > 0) {
     if (X == nullptr || CB == nullptr || SCB == nullptr || Y == nullptr) return I8_ERR_INVALID_ARG;
@@ -135,6 +144,7 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
 
   DevStatus* dst = reinterpret_cast<DevStatus*>(w + L.status);
   uint32_t* mask = reinterpret_cast<uint32_t*>(w + L.mask);
+  uint32_t* prefix = mask + (K + 31) / 32;
   float* sA = reinterpret_cast<float*>(w + L.sA);
   int8_t* Xq = reinterpret_cast<int8_t*>(w + L.Xq);
   __half* Xo = reinterpret_cast<__half*>(w + L.Xo);
@@ -145,11 +155,11 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   if (hb == 0xffffffffu)
     e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
   else
-    e = launch_outliers(Xh, T, K, hb, mask, idx, n_out, dst, stream);
+    e = launch_outliers(Xh, T, K, hb, mask, prefix, idx, n_out, dst, stream);
   if (e != cudaSuccess || !mark(1)) return I8_ERR_CUDA;
 
-  const bool gemv = (path == 2) || (path == 0 && T <= kDecodeMaxT);
-  e = launch_rowquant(Xh, T, K, mask, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, stream);
+  const bool gemv = (path == kPathDecode) || (path == kPathAuto && T <= kDecodeMaxT);
+  e = launch_rowquant(Xh, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, num_sms, stream);
   if (e != cudaSuccess || !mark(2)) return I8_ERR_CUDA;
 
   GemmArgs a;
@@ -170,7 +180,7 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   a.N = N;
   a.K = K;
   a.mode = 0;
-  e = gemv ? launch_gemv_decode(a, num_sms, stream) : launch_gemm_tc(a, num_sms, stream);
+  e = launch_product(a, path, gemv, num_sms, stream);
   if (e != cudaSuccess || !mark(3)) return I8_ERR_CUDA;
   return I8_OK;
 }
@@ -292,8 +302,8 @@ i8_status int8_linear_forward_host(const void* X_host, int64_t T, int64_t K, con
 
 i8_status int8_gemm_i32(const int8_t* Xq, int64_t T, int64_t K, const int8_t* CB, int64_t N, int32_t* acc, int path,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  if (!shape_ok(T, K, N) || path < 0 || path > 2) return I8_ERR_INVALID_ARG;
-  if (path == 2 && T > kDecodeMaxT) return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K, N) || path < kPathAuto || path > kPathTensorCoreSingleSM) return I8_ERR_INVALID_ARG;
+  if (path == kPathDecode && T > kDecodeMaxT) return I8_ERR_INVALID_ARG;
   if (T > 0 && (Xq == nullptr || CB == nullptr || acc == nullptr)) return I8_ERR_INVALID_ARG;
   if (T > 0 && (!aligned(Xq, 16) || !aligned(CB, 16) || !aligned(acc, 16))) return I8_ERR_INVALID_ARG;
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < sizeof(DevStatus)) return I8_ERR_WORKSPACE;
@@ -312,8 +322,8 @@ i8_status int8_gemm_i32(const int8_t* Xq, int64_t T, int64_t K, const int8_t* CB
   a.N = N;
   a.K = K;
   a.mode = 1;
-  const bool gemv = (path == 2) || (path == 0 && T <= kDecodeMaxT);
-  return cuda_status(gemv ? launch_gemv_decode(a, num_sms, stream) : launch_gemm_tc(a, num_sms, stream));
+  const bool gemv = (path == kPathDecode) || (path == kPathAuto && T <= kDecodeMaxT);
+  return cuda_status(launch_product(a, path, gemv, num_sms, stream));
 }
 
 }  // extern "C"

@@ -1,0 +1,413 @@
+// Prefill GEMM of the LLM.int8() forward linear layer, pair-of-SMs version.
+//
+// Same computation as gemm_tc.cu (int8 product over the non-outlier columns,
+// fp16 product over the outlier columns, dequantise with the row and column
+// absmax constants and add the bias: steps 2-3 of "Core idea of LLM.int8()" on
+// the Hugging Face integration page), with the output tile of a 2-CTA cluster
+// computed by one tcgen05.mma.cta_group::2 of M=256, N=256:
+//   * CTA r of the pair holds rows [128r, 128r+128) of the A tile and rows
+//     [128r, 128r+128) of the B tile (B is split along N between the CTAs),
+//     so each SM streams 32 KB per 128-byte K-block instead of 48 KB;
+//   * each CTA's TMEM holds its 128 output rows x 256 columns;
+//   * the even CTA (leader) issues the MMAs; both CTAs' TMA loads complete on
+//     the leader's "full" barrier, and the leader's commits arrive on both
+//     CTAs' "empty" and "TMEM full" barriers;
+//   * both CTAs' epilogues arrive on the leader's "TMEM empty" barrier.
+// No TMA load uses cluster multicast: each CTA loads its own halves.
+#include <cuda.h>
+
+#include "kernels.h"
+
+namespace i8mp {
+namespace {
+
+constexpr int BM = 128;           // rows per CTA (256 per pair)
+constexpr int BN = 256;           // output columns per tile
+constexpr int BN_HALF = BN / 2;   // B rows loaded per CTA
+constexpr int BKB = 128;          // bytes of K per stage
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BKB;       // 16 KB
+constexpr int B_BYTES = BN_HALF * BKB;  // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int THREADS = 64 + NUM_EPI_WARPS * 32;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+constexpr int GROUP_M = 8;  // pair tiles (256 rows) per raster group
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t IDESC_I8 = idesc_i8_s32(2 * BM, BN);
+constexpr uint32_t IDESC_F16 = idesc_f16_f32(2 * BM, BN);
+constexpr uint16_t PAIR_MASK = 0x3;
+
+constexpr uint32_t W_EMPTY = 0x201, W_FULL = 0x202, W_TEMPTY = 0x203, W_TFULL = 0x204, W_DRAIN = 0x205,
+                   W_TEARDOWN = 0x206;
+
+struct Params {
+  int64_t T, N, K;
+  int nkb_i8;
+  const float* sA;
+  const float* SCB;
+  const __half* bias;
+  __half* Y;
+  int32_t* acc_out;
+  const int32_t* n_out;
+  DevStatus* st;
+  int mode;
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
+  const int group_size = GROUP_M * num_n;
+  const int g = tile / group_size;
+  const int first_m = g * GROUP_M;
+  const int gm = min(num_m - first_m, GROUP_M);
+  const int local = tile - g * group_size;
+  m_blk = first_m + local % gm;
+  n_blk = local / gm;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_i8_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmAo, const __grid_constant__ CUtensorMap tmBo,
+                       const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];   // used in the leader only
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];      // used in the leader only
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+
+  const int num_m = static_cast<int>((p.T + 2 * BM - 1) / (2 * BM));
+  const int num_n = static_cast<int>((p.N + BN - 1) / BN);
+  const int num_tiles = num_m * num_n;
+  const int n_out = (p.n_out != nullptr) ? *p.n_out : 0;
+  const int nkb_o = (p.mode == 0) ? (n_out + 63) / 64 : 0;
+  const int nkb = p.nkb_i8 + nkb_o;
+  const bool has_out = nkb_o > 0;
+  const int nbuf = has_out ? 1 : 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 2 * NUM_EPI_WARPS);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (has_out) {
+      tma_prefetch_desc(&tmAo);
+      tma_prefetch_desc(&tmBo);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tmem_base_sh, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int issued[STAGES];
+      #pragma unroll
+      for (int i = 0; i < STAGES; ++i) issued[i] = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        int m_blk, n_blk;
+        tile_coords(tile, num_m, num_n, m_blk, n_blk);
+        const int row_a = m_blk * 2 * BM + static_cast<int>(rank) * BM;
+        const int row_b = n_blk * BN + static_cast<int>(rank) * BN_HALF;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u, &abort_sh, p.st, W_EMPTY)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * STAGE_BYTES);
+          const uint32_t fb = leader_smem_addr(smem_u32(&full_bar[s]));
+          if (kb < p.nkb_i8) {
+            tma_load_2d_pair(sa, &tmA, fb, kb * BKB, row_a);
+            tma_load_2d_pair(sb, &tmB, fb, kb * BKB, row_b);
+          } else {
+            const int ko = kb - p.nkb_i8;
+            tma_load_2d_pair(sa, &tmAo, fb, ko * 64, row_a);
+            tma_load_2d_pair(sb, &tmBo, fb, ko * 64, row_b);
+          }
+          ++issued[s];
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      // The leader's full barriers count both CTAs' loads: once every armed
+      // phase has completed, no load of either CTA is still in flight.
+      if (leader) {
+        for (int i = 0; i < STAGES; ++i) {
+          if (issued[i] > 0) {
+            volatile int never = 0;
+            mbar_wait(&full_bar[i], static_cast<uint32_t>((issued[i] - 1) & 1), &never, p.st, W_TEARDOWN);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (leader only)
+    if (leader && lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++it) {
+        const int buf = it % nbuf;
+        const uint32_t aph = static_cast<uint32_t>((it / nbuf) & 1);
+        if (!mbar_wait_cluster(&tempty_bar[buf], aph ^ 1u, &abort_sh, p.st, W_TEMPTY)) break;
+        tc_fence_after();
+        const uint32_t d_i32 = tmem_base + static_cast<uint32_t>(buf) * 256u;
+        const uint32_t d_f32 = tmem_base + 256u;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full_bar[s], ph, &abort_sh, p.st, W_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+          const uint64_t adesc = sw128_kmajor_desc(a_addr);
+          const uint64_t bdesc = sw128_kmajor_desc(a_addr + A_BYTES);
+          if (kb < p.nkb_i8) {
+            #pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_i8_pair(d_i32, adesc + 2u * kk, bdesc + 2u * kk, IDESC_I8, (kb | kk) != 0 ? 1u : 0u);
+          } else {
+            const int ko = kb - p.nkb_i8;
+            #pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_pair(d_f32, adesc + 2u * kk, bdesc + 2u * kk, IDESC_F16, (ko | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit_pair(&empty_bar[s], PAIR_MASK);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (ok) mma_commit_pair(&tfull_bar[buf], PAIR_MASK);
+      }
+      mma_commit_pair(&drain_bar, 0x1);
+      volatile int never = 0;
+      mbar_wait(&drain_bar, 0u, &never, p.st, W_DRAIN);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    int it = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+      const int buf = it % nbuf;
+      const uint32_t aph = static_cast<uint32_t>((it / nbuf) & 1);
+      int m_blk, n_blk;
+      tile_coords(tile, num_m, num_n, m_blk, n_blk);
+      if (!mbar_wait_cluster(&tfull_bar[buf], aph, &abort_sh, p.st, W_TFULL)) break;
+      tc_fence_after();
+      const int64_t row = static_cast<int64_t>(m_blk) * 2 * BM + static_cast<int64_t>(rank) * BM + q * 32 + lane;
+      const bool row_ok = row < p.T;
+      const float ra = (row_ok && p.mode == 0) ? __ldg(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
+      #pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        const int col0 = half * 128 + c * 32;
+        const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
+        uint32_t acc[32];
+        uint32_t fo[32];
+        tmem_ld_32x32b_x32(tmem_base + lane_base + static_cast<uint32_t>(buf) * 256u + col0, acc);
+        if (has_out) tmem_ld_32x32b_x32(tmem_base + lane_base + 256u + col0, fo);
+        tmem_ld_wait();
+        if (p.mode == 1) {
+          if (row_ok) {
+            int32_t* dst = p.acc_out + row * p.N + gcol0;
+            #pragma unroll
+            for (int g = 0; g < 8; ++g)
+              if (gcol0 + g * 4 + 4 <= p.N)
+                reinterpret_cast<int4*>(dst)[g] = make_int4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]);
+          }
+          continue;
+        }
+        const int64_t my_col = gcol0 + lane;
+        const float scb_l = (my_col < p.N) ? __ldg(&p.SCB[my_col]) : 0.0f;
+        const float b_l = (p.bias != nullptr && my_col < p.N) ? __half2float(p.bias[my_col]) : 0.0f;
+        uint32_t packed[16];
+        #pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float s0 = __shfl_sync(0xffffffffu, scb_l, i);
+          const float s1 = __shfl_sync(0xffffffffu, scb_l, i + 1);
+          const float b0 = __shfl_sync(0xffffffffu, b_l, i);
+          const float b1 = __shfl_sync(0xffffffffu, b_l, i + 1);
+          float y0 = static_cast<float>(static_cast<int32_t>(acc[i])) * (ra * s0) + b0;
+          float y1 = static_cast<float>(static_cast<int32_t>(acc[i + 1])) * (ra * s1) + b1;
+          if (has_out) {
+            y0 += __uint_as_float(fo[i]);
+            y1 += __uint_as_float(fo[i + 1]);
+          }
+          packed[i >> 1] = pack_half2(y0, y1);
+        }
+        if (row_ok) {
+          __half* dst = p.Y + row * p.N + gcol0;
+          #pragma unroll
+          for (int g = 0; g < 4; ++g)
+            if (gcol0 + g * 8 + 8 <= p.N)
+              reinterpret_cast<uint4*>(dst)[g] =
+                  make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(&tempty_bar[buf], 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the leader's MMAs have drained before either CTA releases TMEM or exits
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode_fn() {
+  static EncodeFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t rows,
+              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows) {
+  EncodeFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int g_max_pairs[64] = {0};
+
+}  // namespace
+
+// Largest number of co-resident 2-CTA clusters of the pair kernel on the
+// current device (0 if clusters of this kernel cannot be launched).
+int pair_kernel_max_clusters() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (g_max_pairs[dev] != 0) return g_max_pairs[dev];
+  if (cudaFuncSetAttribute(gemm_i8_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+      cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_i8_tc2_kernel, &cfg) != cudaSuccess) return 0;
+  g_max_pairs[dev] = n;
+  return n;
+}
+
+cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s) {
+  const int max_pairs = pair_kernel_max_clusters();
+  if (max_pairs <= 0) return cudaErrorNotSupported;
+  if (a.T == 0 || a.N == 0) return cudaSuccess;
+  CUtensorMap tmA, tmB, tmAo, tmBo;
+  if (!make_map(&tmA, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K, a.T, a.K, BKB, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&tmB, a.CB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K, a.N, a.K, BKB, BN_HALF)) return cudaErrorInvalidValue;
+  const bool outl = a.mode == 0 && a.n_out != nullptr && a.Xo != nullptr && a.Wo != nullptr;
+  if (outl) {
+    if (!make_map(&tmAo, a.Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.ldo, a.T, a.ldo * 2, 64, BM))
+      return cudaErrorInvalidValue;
+    if (!make_map(&tmBo, a.Wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.ldo, a.N, a.ldo * 2, 64, BN_HALF))
+      return cudaErrorInvalidValue;
+  } else {
+    tmAo = tmA;
+    tmBo = tmB;
+  }
+  Params p;
+  p.T = a.T;
+  p.N = a.N;
+  p.K = a.K;
+  p.nkb_i8 = static_cast<int>((a.K + BKB - 1) / BKB);
+  p.sA = a.sA;
+  p.SCB = a.SCB;
+  p.bias = a.bias;
+  p.Y = a.Y;
+  p.acc_out = a.acc_out;
+  p.n_out = outl ? a.n_out : nullptr;
+  p.st = a.st;
+  p.mode = a.mode;
+  const int64_t tiles = ((a.T + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
+  if (tiles > 0x3fffffff) return cudaErrorInvalidValue;
+  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_i8_tc2_kernel, tmA, tmB, tmAo, tmBo, p);
+}
+
+}  // namespace i8mp

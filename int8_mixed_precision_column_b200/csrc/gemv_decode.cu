@@ -12,9 +12,13 @@
 // Fragment trick: the dot product is a sum over k, so any permutation of k
 // applied to both operands leaves it unchanged.  Thread (g, t) of a warp loads
 // 16 contiguous bytes of weight row g at k0 + 16t and the same 16 bytes of
-// token rows g and g+8; two MMAs consume them (bytes 0-7, then 8-15).
+// token rows g and g+8; two MMAs consume them (bytes 0-7, then 8-15).  Every
+// thread issues the weight loads of two K-steps for all 4 row groups before
+// its first MMA, so 8 x 16 bytes per thread are in flight.
 // Epilogue: Y = fp16(acc * sA[t] * SCB[j] / 127^2 + sum_o Xo[t,o] * Wo[j,o] + b[j])
-// with Wo[j,o] = fp16((CB[j, idx[o]] * SCB[j]) / 127) recomputed from CB.
+// with Wo[j,o] = fp16((CB[j, idx[o]] * SCB[j]) / 127) recomputed from CB; the
+// outlier operands of a 32-row chunk are staged in shared memory, 64 outlier
+// columns at a time.
 #include "kernels.h"
 
 namespace i8mp {
@@ -22,7 +26,9 @@ namespace {
 
 constexpr int DV_WARPS = 8;
 constexpr int DV_THREADS = DV_WARPS * 32;
-constexpr int DV_RG = 4;  // 8-row groups per pass
+constexpr int DV_RG = 4;   // 8-row groups per pass (32 rows)
+constexpr int DV_U = 2;    // K-steps (64 B each) loaded before computing
+constexpr int DV_OB = 64;  // outlier columns staged per block
 
 struct DvParams {
   const int8_t* Xq;
@@ -57,8 +63,10 @@ __device__ __forceinline__ uint4 ld_stream(const int8_t* p) {
   return v;
 }
 
-__global__ void __launch_bounds__(DV_THREADS) gemv_i8_decode_kernel(const DvParams p) {
+__global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvParams p) {
   __shared__ int32_t red[DV_WARPS][DV_RG][32][4];
+  __shared__ float wo_s[DV_RG * 8][DV_OB + 1];
+  __shared__ float xo_s[kDecodeMaxT][DV_OB + 1];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;
@@ -74,6 +82,7 @@ __global__ void __launch_bounds__(DV_THREADS) gemv_i8_decode_kernel(const DvPara
   const bool row_b = g + 8 < p.T;
   const int8_t* xa_base = p.Xq + static_cast<int64_t>(g) * p.K + t4 * 16;
   const int8_t* xb_base = p.Xq + static_cast<int64_t>(g + 8) * p.K + t4 * 16;
+  const uint4 zero4 = make_uint4(0, 0, 0, 0);
 
   for (int64_t g0 = g_begin; g0 < g_end; g0 += DV_RG) {
     int32_t c[DV_RG][4];
@@ -86,19 +95,31 @@ __global__ void __launch_bounds__(DV_THREADS) gemv_i8_decode_kernel(const DvPara
       wok[r] = (g0 + r) < g_end;
       wrow[r] = p.CB + ((g0 + r) * 8 + g) * p.K + t4 * 16;
     }
-    #pragma unroll 2
-    for (int64_t st = s_begin; st < s_end; ++st) {
-      const int64_t k = st * 64;
-      const bool kok = k + t4 * 16 < p.K;
-      uint4 w[DV_RG];
+    #pragma unroll 1
+    for (int64_t st = s_begin; st < s_end; st += DV_U) {
+      uint4 w[DV_U][DV_RG];
+      uint4 xa[DV_U], xb[DV_U];
       #pragma unroll
-      for (int r = 0; r < DV_RG; ++r) w[r] = (wok[r] && kok) ? ld_stream(wrow[r] + k) : make_uint4(0, 0, 0, 0);
-      const uint4 xa = (row_a && kok) ? __ldg(reinterpret_cast<const uint4*>(xa_base + k)) : make_uint4(0, 0, 0, 0);
-      const uint4 xb = (row_b && kok) ? __ldg(reinterpret_cast<const uint4*>(xb_base + k)) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < DV_U; ++u) {
+        const int64_t k = (st + u) * 64;
+        const bool kok = (st + u) < s_end && k + t4 * 16 < p.K;
+        #pragma unroll
+        for (int r = 0; r < DV_RG; ++r) w[u][r] = (wok[r] && kok) ? ld_stream(wrow[r] + k) : zero4;
+      }
       #pragma unroll
-      for (int r = 0; r < DV_RG; ++r) {
-        mma_s8_16832(c[r], xa.x, xb.x, xa.y, xb.y, w[r].x, w[r].y);
-        mma_s8_16832(c[r], xa.z, xb.z, xa.w, xb.w, w[r].z, w[r].w);
+      for (int u = 0; u < DV_U; ++u) {
+        const int64_t k = (st + u) * 64;
+        const bool kok = (st + u) < s_end && k + t4 * 16 < p.K;
+        xa[u] = (row_a && kok) ? __ldg(reinterpret_cast<const uint4*>(xa_base + k)) : zero4;
+        xb[u] = (row_b && kok) ? __ldg(reinterpret_cast<const uint4*>(xb_base + k)) : zero4;
+      }
+      #pragma unroll
+      for (int u = 0; u < DV_U; ++u) {
+        #pragma unroll
+        for (int r = 0; r < DV_RG; ++r) {
+          mma_s8_16832(c[r], xa[u].x, xb[u].x, xa[u].y, xb[u].y, w[u][r].x, w[u][r].y);
+          mma_s8_16832(c[r], xa[u].z, xb[u].z, xa[u].w, xb[u].w, w[u][r].z, w[u][r].w);
+        }
       }
     }
     #pragma unroll
@@ -107,33 +128,66 @@ __global__ void __launch_bounds__(DV_THREADS) gemv_i8_decode_kernel(const DvPara
       for (int i = 0; i < 4; ++i) red[warp][r][lane][i] = c[r][i];
     }
     __syncthreads();
-    // 4 groups x 32 lanes x 4 values = 512 outputs (token, row) per pass.
-    for (int v = threadIdx.x; v < DV_RG * 128; v += DV_THREADS) {
+
+    // Each thread owns two (token, row) outputs of the 512 this pass produces.
+    int32_t acc[2];
+    float yo[2] = {0.0f, 0.0f};
+    int tok[2], jr[2];
+    bool live[2];
+    #pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int v = threadIdx.x + h * DV_THREADS;
       const int r = v >> 7;
       const int ln = (v >> 2) & 31;
       const int i = v & 3;
-      if (g0 + r >= g_end) continue;
-      const int tok = (ln >> 2) + ((i >> 1) << 3);
-      if (tok >= p.T) continue;
-      const int64_t j = (g0 + r) * 8 + (ln & 3) * 2 + (i & 1);
-      int32_t acc = 0;
+      tok[h] = (ln >> 2) + ((i >> 1) << 3);
+      jr[h] = r * 8 + (ln & 3) * 2 + (i & 1);
+      live[h] = (g0 + r < g_end) && tok[h] < p.T;
+      int32_t s = 0;
       #pragma unroll
-      for (int w = 0; w < DV_WARPS; ++w) acc += red[w][r][ln][i];
+      for (int w = 0; w < DV_WARPS; ++w) s += red[w][r][ln][i];
+      acc[h] = s;
+    }
+    // 16-bit product over the outlier columns, DV_OB columns at a time.
+    for (int ob = 0; ob < n_out; ob += DV_OB) {
+      const int nb = min(DV_OB, n_out - ob);
+      for (int e = threadIdx.x; e < DV_RG * 8 * nb; e += DV_THREADS) {
+        const int r = e / nb;
+        const int o = e - r * nb;
+        const int64_t j = g0 * 8 + r;
+        float wv = 0.0f;
+        if (j < g_end * 8) {
+          const float cbv = static_cast<float>(__ldg(&p.CB[j * p.K + __ldg(&p.idx[ob + o])]));
+          wv = __half2float(__float2half_rn(__fdiv_rn(__fmul_rn(cbv, __ldg(&p.SCB[j])), 127.0f)));
+        }
+        wo_s[r][o] = wv;
+      }
+      for (int e = threadIdx.x; e < kDecodeMaxT * nb; e += DV_THREADS) {
+        const int t = e / nb;
+        const int o = e - t * nb;
+        xo_s[t][o] = (t < p.T) ? __half2float(p.Xo[t * p.ldo + ob + o]) : 0.0f;
+      }
+      __syncthreads();
+      #pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float s = yo[h];
+        for (int o = 0; o < nb; ++o) s = fmaf(xo_s[tok[h]][o], wo_s[jr[h]][o], s);
+        yo[h] = s;
+      }
+      __syncthreads();
+    }
+    #pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (!live[h]) continue;
+      const int64_t j = g0 * 8 + jr[h];
       if (p.mode == 1) {
-        p.acc_out[tok * p.N + j] = acc;
+        p.acc_out[tok[h] * p.N + j] = acc[h];
         continue;
       }
       const float scb = __ldg(&p.SCB[j]);
-      float y = static_cast<float>(acc) * (__ldg(&p.sA[tok]) * (1.0f / 16129.0f) * scb);
-      float yo = 0.0f;
-      for (int o = 0; o < n_out; ++o) {
-        const float cbv = static_cast<float>(__ldg(&p.CB[j * p.K + __ldg(&p.idx[o])]));
-        const float wo = __half2float(__float2half_rn(__fdiv_rn(__fmul_rn(cbv, scb), 127.0f)));
-        yo = fmaf(__half2float(p.Xo[tok * p.ldo + o]), wo, yo);
-      }
-      y += yo;
+      float y = static_cast<float>(acc[h]) * (__ldg(&p.sA[tok[h]]) * (1.0f / 16129.0f) * scb) + yo[h];
       if (p.bias != nullptr) y += __half2float(p.bias[j]);
-      p.Y[tok * p.N + j] = __float2half_rn(y);
+      p.Y[tok[h] * p.N + j] = __float2half_rn(y);
     }
     __syncthreads();
   }

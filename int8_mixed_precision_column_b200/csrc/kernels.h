@@ -17,16 +17,17 @@ cudaError_t launch_quantize_weight(const __half* W, int64_t N, int64_t K, int8_t
 // Column outlier mask (atomicOr into a zeroed mask) followed, in the last CTA
 // to finish, by compaction into the ascending idx list and n_out.
 // `hbits` is the largest fp16 magnitude bit pattern whose value is <= threshold.
+// Also writes prefix[w] = number of outlier columns in mask words 0..w-1.
 cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
-                            int32_t* idx, int32_t* n_out, DevStatus* st, cudaStream_t s);
+                            uint32_t* prefix, int32_t* idx, int32_t* n_out, DevStatus* st, cudaStream_t s);
 
 // Row-wise absmax int8 quantisation over non-outlier columns, fp16 gather of
 // the outlier activation columns into Xo, and (when `with_wo`) the gather and
 // dequantisation of the matching weight columns into Wo.
-cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_t* mask, const int32_t* idx,
-                            const int32_t* n_out, int8_t* Xq, float* sA, __half* Xo, int64_t ldo,
-                            const int8_t* CB, const float* SCB, int64_t N, __half* Wo, bool with_wo,
-                            cudaStream_t s);
+cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_t* mask, const uint32_t* prefix,
+                            const int32_t* idx, const int32_t* n_out, int8_t* Xq, float* sA, __half* Xo,
+                            int64_t ldo, const int8_t* CB, const float* SCB, int64_t N, __half* Wo, bool with_wo,
+                            int num_sms, cudaStream_t s);
 
 struct GemmArgs {
   const int8_t* Xq;      // [T,K]
@@ -50,10 +51,19 @@ struct GemmArgs {
 // kind::f16 outlier product and dequant/bias epilogue.
 cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t s);
 
+// Prefill, pair-of-SMs version: 2-CTA clusters, tcgen05.mma.cta_group::2 with
+// 256 x 256 tiles.  Returns cudaErrorNotSupported if such clusters cannot be
+// launched on the current device.
+cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s);
+int pair_kernel_max_clusters();
+
 // Decode (T <= 16): weight-streaming int8 GEMV on mma.sync with the outlier
 // columns dequantised from CB in the epilogue.
 cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s);
 
 constexpr int kDecodeMaxT = 16;
+
+// Product-kernel choice (the `path` argument of the C ABI).
+enum Path : int { kPathAuto = 0, kPathTensorCore = 1, kPathDecode = 2, kPathTensorCoreSingleSM = 3 };
 
 }  // namespace i8mp

@@ -15,7 +15,7 @@
 // It runs the same kernels as int8_linear_forward's decode path (T <= 16).
 #include <mutex>
 
-#include "../../include/int8mp.h"
+#include "int8mp.h"
 #include "kernels.h"
 
 using namespace i8mp;
@@ -42,7 +42,7 @@ StaticLayout static_layout(int64_t T, int64_t K) {
   L.ldo = ((K + 63) / 64) * 64;
   L.status = 0;
   L.mask = 256;
-  L.sA = up256(L.mask + static_cast<uint64_t>((K + 31) / 32) * 4);
+  L.sA = up256(L.mask + static_cast<uint64_t>((K + 31) / 32) * 8);  // mask words + prefix counts
   L.Xq = up256(L.sA + static_cast<uint64_t>(T) * 4);
   L.Xo = up256(L.Xq + static_cast<uint64_t>(T) * K);
   L.total = up256(L.Xo + static_cast<uint64_t>(T) * L.ldo * 2);
@@ -111,9 +111,10 @@ extern "C" i8_status int8_linear_forward_decode_static(const void* X, int64_t T,
   if (hb == 0xffffffffu)
     e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
   else
-    e = launch_outliers(Xh, T, K, hb, mask, idx, n_out, dst, stream);
+    e = launch_outliers(Xh, T, K, hb, mask, mask + (K + 31) / 32, idx, n_out, dst, stream);
   if (e != cudaSuccess) return I8_ERR_CUDA;
-  e = launch_rowquant(Xh, T, K, mask, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, nullptr, false, stream);
+  e = launch_rowquant(Xh, T, K, mask, mask + (K + 31) / 32, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, nullptr,
+                      false, num_sms, stream);
   if (e != cudaSuccess) return I8_ERR_CUDA;
 
   GemmArgs a;

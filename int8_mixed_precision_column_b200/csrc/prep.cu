@@ -65,7 +65,9 @@ cudaError_t launch_quantize_weight(const __half* W, int64_t N, int64_t K, int8_t
 // the largest pattern whose value is <= threshold (computed on the host).
 // NaN patterns (> 0x7c00) are excluded so that NaN never flags a column.
 // The CTA merges its 8 warps in shared memory and ORs 8 words into the mask.
-// The last CTA to finish compacts the mask into the ascending idx list.
+// The last CTA to finish compacts the mask into the ascending idx list and
+// records, per mask word, how many outlier columns precede it (prefix), so
+// that the rank of an outlier column is prefix[w] + popc(lower bits of word w).
 // ---------------------------------------------------------------------------
 constexpr int kMaskThreads = 256;
 constexpr int kMaskRowsPerChunk = 128;
@@ -84,8 +86,8 @@ __device__ __forceinline__ uint32_t flag_bits8(const uint4& v, uint32_t h2) {
 
 __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const __half* __restrict__ X, int64_t T, int64_t K,
                                                                     uint32_t hbits, uint32_t* __restrict__ mask,
-                                                                    int32_t* __restrict__ idx, int32_t* __restrict__ n_out,
-                                                                    DevStatus* st) {
+                                                                    uint32_t* __restrict__ prefix, int32_t* __restrict__ idx,
+                                                                    int32_t* __restrict__ n_out, DevStatus* st) {
   __shared__ uint32_t s_words[8];
   __shared__ int s_last;
   __shared__ int s_scan[kMaskThreads];
@@ -149,6 +151,7 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const __half
   int pos = s_scan[threadIdx.x] - cnt;
   for (int64_t w = w0; w < w1; ++w) {
     uint32_t m = __ldcg(&mask[w]);
+    prefix[w] = static_cast<uint32_t>(pos);
     while (m) {
       const int b = __ffs(m) - 1;
       m &= m - 1;
@@ -161,13 +164,13 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const __half
   }
 }
 
-cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask, int32_t* idx,
-                            int32_t* n_out, DevStatus* st, cudaStream_t s) {
+cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
+                            uint32_t* prefix, int32_t* idx, int32_t* n_out, DevStatus* st, cudaStream_t s) {
   const int64_t slabs = (K + 255) / 256;
   const int64_t chunks = (T + kMaskRowsPerChunk - 1) / kMaskRowsPerChunk;
   if (slabs > 0x7fffffff || chunks > 65535) return cudaErrorInvalidValue;
   dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(chunks));
-  outlier_mask_kernel<<<grid, kMaskThreads, 0, s>>>(X, T, K, hbits, mask, idx, n_out, st);
+  outlier_mask_kernel<<<grid, kMaskThreads, 0, s>>>(X, T, K, hbits, mask, prefix, idx, n_out, st);
   return cudaGetLastError();
 }
 
@@ -176,15 +179,17 @@ cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbit
 //
 // Blocks [0, T): one CTA per token row t.  The row is read once into registers
 // (8 columns per 16-byte chunk), the absmax over non-outlier columns is
-// reduced across the CTA, and the codes are written as 8-byte packets.  The
-// CTA then writes the row of Xo: X[t, idx[o]] for o < n_out, zero up to the
-// next multiple of 64 (the K-block of the fp16 outlier MMA).
-// Blocks [T, T + ceil(N/kWoRows)): rows of Wo = fp16((CB[j, idx[o]] * SCB[j]) / 127),
-// zero-padded the same way (only when the tensor-core path consumes Wo).
+// reduced across the CTA, and the codes are written as 8-byte packets.  Each
+// outlier value goes from registers straight to Xo[t, rank], its rank among
+// the outlier columns being prefix[word] + popc(lower bits of the word); Xo is
+// zero-padded to the next multiple of 64 (the K-block of the fp16 outlier MMA).
+// Blocks [T, ...): Wo[j, o] = fp16((CB[j, idx[o]] * SCB[j]) / 127) with the
+// same padding (only when the tensor-core path consumes Wo), four independent
+// gathers per thread in flight.
 // ---------------------------------------------------------------------------
 constexpr int kRowThreads = 256;
 constexpr int kRowChunks = 8;   // registers hold rows up to 256*8*8 = 16384 columns
-constexpr int kWoRows = 32;
+constexpr int kWoUnroll = 4;
 
 __device__ __forceinline__ uint32_t mask_byte(const uint32_t* mask, int64_t chunk) {
   return (__ldg(&mask[chunk >> 2]) >> ((chunk & 3) * 8)) & 0xffu;
@@ -210,11 +215,24 @@ __device__ __forceinline__ uint2 row_codes(const uint4& v, uint32_t mb, float in
   return make_uint2(w[0], w[1]);
 }
 
-__global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
+// Scatter the outlier entries of one 8-column chunk into the Xo row.
+__device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, int64_t chunk, const uint32_t* mask,
+                                                 const uint32_t* prefix, __half* xo_row) {
+  const __half* h = reinterpret_cast<const __half*>(&v);
+  const uint32_t mw = __ldg(&mask[chunk >> 2]);
+  const uint32_t base = __ldg(&prefix[chunk >> 2]);
+  const int sh = static_cast<int>(chunk & 3) * 8;
+  #pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if ((mb >> e) & 1u) xo_row[base + __popc(mw & ((1u << (sh + e)) - 1u))] = h[e];
+}
+
+__global__ void __launch_bounds__(kRowThreads, 3) rowquant_kernel(
     const __half* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
-    const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p, int8_t* __restrict__ Xq,
-    float* __restrict__ sA, __half* __restrict__ Xo, int64_t ldo, const int8_t* __restrict__ CB,
-    const float* __restrict__ SCB, int64_t N, __half* __restrict__ Wo, int with_wo) {
+    const uint32_t* __restrict__ prefix, const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p,
+    int8_t* __restrict__ Xq, float* __restrict__ sA, __half* __restrict__ Xo, int64_t ldo,
+    const int8_t* __restrict__ CB, const float* __restrict__ SCB, int64_t N, __half* __restrict__ Wo,
+    int64_t wo_blocks) {
   __shared__ float s_red[kRowThreads / 32];
   const int tid = threadIdx.x;
   const int n_out = *n_out_p;
@@ -222,19 +240,30 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
 
   if (static_cast<int64_t>(blockIdx.x) >= T) {
     // ---- Wo rows ----
-    if (!with_wo || n_out == 0) return;
-    const int64_t j0 = (static_cast<int64_t>(blockIdx.x) - T) * kWoRows;
-    const int64_t total = static_cast<int64_t>(kWoRows) * npad;
-    for (int64_t e = tid; e < total; e += kRowThreads) {
-      const int64_t j = j0 + e / npad;
-      const int64_t o = e % npad;
-      if (j >= N) break;
-      __half v = __float2half_rn(0.0f);
-      if (o < n_out) {
-        const float c = static_cast<float>(__ldg(&CB[j * K + __ldg(&idx[o])]));
-        v = __float2half_rn(__fdiv_rn(__fmul_rn(c, __ldg(&SCB[j])), 127.0f));
+    if (n_out == 0) return;
+    const int64_t total = N * npad;
+    const int64_t stride = wo_blocks * kRowThreads * kWoUnroll;
+    for (int64_t e0 = (static_cast<int64_t>(blockIdx.x) - T) * kRowThreads * kWoUnroll + tid; e0 < total;
+         e0 += stride) {
+      int8_t cbv[kWoUnroll];
+      int64_t jj[kWoUnroll], oo[kWoUnroll];
+      #pragma unroll
+      for (int u = 0; u < kWoUnroll; ++u) {
+        const int64_t e = e0 + static_cast<int64_t>(u) * kRowThreads;
+        jj[u] = e / npad;
+        oo[u] = e - jj[u] * npad;
+        cbv[u] = (e < total && oo[u] < n_out) ? __ldg(&CB[jj[u] * K + __ldg(&idx[oo[u]])]) : int8_t(0);
       }
-      Wo[j * ldo + o] = v;
+      #pragma unroll
+      for (int u = 0; u < kWoUnroll; ++u) {
+        const int64_t e = e0 + static_cast<int64_t>(u) * kRowThreads;
+        if (e < total) {
+          __half v = __float2half_rn(0.0f);
+          if (oo[u] < n_out)
+            v = __float2half_rn(__fdiv_rn(__fmul_rn(static_cast<float>(cbv[u]), __ldg(&SCB[jj[u]])), 127.0f));
+          Wo[jj[u] * ldo + oo[u]] = v;
+        }
+      }
     }
     return;
   }
@@ -270,30 +299,40 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
   const float inv = scale_inv(absmax);
   if (tid == 0) sA[t] = absmax;
   uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
+  __half* xo_row = Xo + t * ldo;
   #pragma unroll
   for (int c = 0; c < kRowChunks; ++c) {
     const int64_t i = tid + static_cast<int64_t>(c) * kRowThreads;
-    if (i < nv) dst[i] = row_codes(v[c], mb[c], inv);
+    if (i < nv) {
+      dst[i] = row_codes(v[c], mb[c], inv);
+      if (mb[c]) scatter_outliers(v[c], mb[c], i, mask, prefix, xo_row);
+    }
   }
-  for (int64_t i = tid + static_cast<int64_t>(kRowChunks) * kRowThreads; i < nv; i += kRowThreads)
-    dst[i] = row_codes(__ldg(src + i), mask_byte(mask, i), inv);
-
-  if (n_out > 0) {
-    const __half* xrow = X + t * K;
-    for (int64_t o = tid; o < npad; o += kRowThreads)
-      Xo[t * ldo + o] = (o < n_out) ? xrow[__ldg(&idx[o])] : __float2half_rn(0.0f);
+  for (int64_t i = tid + static_cast<int64_t>(kRowChunks) * kRowThreads; i < nv; i += kRowThreads) {
+    const uint4 vv = __ldg(src + i);
+    const uint32_t b = mask_byte(mask, i);
+    dst[i] = row_codes(vv, b, inv);
+    if (b) scatter_outliers(vv, b, i, mask, prefix, xo_row);
   }
+  for (int64_t o = n_out + tid; o < npad; o += kRowThreads) xo_row[o] = __float2half_rn(0.0f);
 }
 
-cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_t* mask, const int32_t* idx,
-                            const int32_t* n_out, int8_t* Xq, float* sA, __half* Xo, int64_t ldo, const int8_t* CB,
-                            const float* SCB, int64_t N, __half* Wo, bool with_wo, cudaStream_t s) {
-  const int64_t wo_blocks = with_wo ? (N + kWoRows - 1) / kWoRows : 0;
+cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_t* mask, const uint32_t* prefix,
+                            const int32_t* idx, const int32_t* n_out, int8_t* Xq, float* sA, __half* Xo, int64_t ldo,
+                            const int8_t* CB, const float* SCB, int64_t N, __half* Wo, bool with_wo, int num_sms,
+                            cudaStream_t s) {
+  int64_t wo_blocks = 0;
+  if (with_wo) {
+    wo_blocks = (N * 64 + kRowThreads * kWoUnroll - 1) / (kRowThreads * kWoUnroll);
+    const int64_t cap = static_cast<int64_t>(num_sms) * 4;
+    if (wo_blocks > cap) wo_blocks = cap;
+    if (wo_blocks < 1) wo_blocks = 1;
+  }
   const int64_t blocks = T + wo_blocks;
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
-  rowquant_kernel<<<static_cast<unsigned>(blocks), kRowThreads, 0, s>>>(X, T, K, mask, idx, n_out, Xq, sA, Xo, ldo,
-                                                                        CB, SCB, N, Wo, with_wo ? 1 : 0);
+  rowquant_kernel<<<static_cast<unsigned>(blocks), kRowThreads, 0, s>>>(X, T, K, mask, prefix, idx, n_out, Xq, sA,
+                                                                        Xo, ldo, CB, SCB, N, Wo, wo_blocks);
   return cudaGetLastError();
 }
 

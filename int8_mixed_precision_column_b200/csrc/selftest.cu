@@ -2,7 +2,7 @@
 // single thread waits on an mbarrier that nothing ever arrives on, with a short
 // limit.  The wait must give up, record kErrTimeout with its tag in the
 // workspace status word and return, leaving the CUDA context usable.
-#include "../../include/int8mp.h"
+#include "int8mp.h"
 #include "kernels.h"
 
 using namespace i8mp;

@@ -22,7 +22,7 @@ I8_OK = 0
 STATUS_NAMES = {0: "I8_OK", 1: "I8_ERR_INVALID_ARG", 2: "I8_ERR_WORKSPACE", 3: "I8_ERR_CUDA",
                 4: "I8_ERR_TIMEOUT", 5: "I8_ERR_UNSUPPORTED"}
 
-PATH_AUTO, PATH_TENSOR_CORE, PATH_DECODE = 0, 1, 2
+PATH_AUTO, PATH_TENSOR_CORE, PATH_DECODE, PATH_TENSOR_CORE_1SM = 0, 1, 2, 3
 DECODE_MAX_T = 16
 
 _lib = None

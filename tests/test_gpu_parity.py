@@ -19,7 +19,8 @@ from int8_mixed_precision_column_b200 import build, native, workloads
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"auto": native.PATH_AUTO, "tc": native.PATH_TENSOR_CORE, "decode": native.PATH_DECODE}
+PATHS = {"auto": native.PATH_AUTO, "tc": native.PATH_TENSOR_CORE, "decode": native.PATH_DECODE,
+         "tc1": native.PATH_TENSOR_CORE_1SM}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -132,10 +133,11 @@ RAGGED = [
 ]
 
 
+@pytest.mark.parametrize("path", ["tc", "tc1"])
 @pytest.mark.parametrize("T,K,N,planted,thr", RAGGED)
-def test_ragged_tensor_core(T, K, N, planted, thr):
+def test_ragged_tensor_core(T, K, N, planted, thr, path):
     p = workloads.make_problem("ragged", T, K, N, n_planted=planted, bias_std=0.01, threshold=thr, seed=T + K + N)
-    check_forward(p, gpu_forward(p, "tc"))
+    check_forward(p, gpu_forward(p, path))
 
 
 @pytest.mark.parametrize("T", [1, 2, 5, 8, 9, 15, 16])
@@ -232,8 +234,9 @@ def test_deterministic_repeat():
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("T,K,N,path", [(16, 64, 64, "tc"), (200, 208, 272, "tc"), (384, 1536, 768, "tc"),
-                                        (16, 14336, 512, "tc"), (1, 64, 64, "decode"), (16, 1216, 400, "decode"),
-                                        (7, 14336, 256, "decode")])
+                                        (16, 14336, 512, "tc"), (16, 64, 64, "tc1"), (200, 208, 272, "tc1"),
+                                        (384, 1536, 768, "tc1"), (600, 4096, 1040, "tc"), (1, 64, 64, "decode"),
+                                        (16, 1216, 400, "decode"), (7, 14336, 256, "decode")])
 def test_gemm_i32_bit_exact(T, K, N, path):
     g = torch.Generator().manual_seed(T * 3 + K)
     Xq = torch.randint(-127, 128, (T, K), generator=g, dtype=torch.int8)
@@ -265,12 +268,13 @@ def tile_cols(N, per_tile=8, tile=256):
     return np.unique(np.array(cols))
 
 
-def test_llama7b_prefill_full():
+@pytest.mark.parametrize("path", ["auto", "tc1"])
+def test_llama7b_prefill_full(path):
     p = workloads.llama7b_prefill(seed=0)
-    g = gpu_forward(p, "auto")
+    g = gpu_forward(p, path)
     r = check_forward(p, g)
     assert g["n_out"] == len(p.planted_cols) and r["idx"].tolist() == p.planted_cols
-    acc = native.int8_gemm_i32(g["Xq"], g["CB"], path=native.PATH_TENSOR_CORE)
+    acc = native.int8_gemm_i32(g["Xq"], g["CB"], path=PATHS["tc" if path == "auto" else path])
     assert np.array_equal(to_np(acc), r["acc"])
 
 
