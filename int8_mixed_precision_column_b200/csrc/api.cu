@@ -159,7 +159,10 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   if (e != cudaSuccess || !mark(1)) return I8_ERR_CUDA;
 
   const bool gemv = (path == kPathDecode) || (path == kPathAuto && T <= kDecodeMaxT);
-  e = launch_rowquant(Xh, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, num_sms, stream);
+  // programmatic launches only directly after one of our kernels
+  const bool after_outliers = (hb != 0xffffffffu);
+  e = launch_rowquant(Xh, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, num_sms, dst,
+                      after_outliers, stream);
   if (e != cudaSuccess || !mark(2)) return I8_ERR_CUDA;
 
   GemmArgs a;
@@ -180,6 +183,7 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   a.N = N;
   a.K = K;
   a.mode = 0;
+  a.pdl = true;  // follows the row quantisation kernel
   e = launch_product(a, path, gemv, num_sms, stream);
   if (e != cudaSuccess || !mark(3)) return I8_ERR_CUDA;
   return I8_OK;

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int num_m = static_cast<int>((p.T + BM - 1) / BM);
   const int num_n = static_cast<int>((p.N + BN - 1) / BN);
   const int num_tiles = num_m * num_n;
+  griddep_wait();  // n_out and the operands come from the preceding kernels
   const int n_out = (p.n_out != nullptr) ? *p.n_out : 0;
   const int nkb_o = (p.mode == 0) ? (n_out + 63) / 64 : 0;
   const int nkb = p.nkb_i8 + nkb_o;
@@ -375,8 +376,17 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t s) {
   const int64_t tiles = ((a.T + BM - 1) / BM) * ((a.N + BN - 1) / BN);
   if (tiles > 0x7fffffff) return cudaErrorInvalidValue;
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  gemm_i8_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmAo, tmBo, p);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel, tmA, tmB, tmAo, tmBo, p);
 }
 
 }  // namespace i8mp

@@ -13,6 +13,9 @@
 //     the leader's "full" barrier, and the leader's commits arrive on both
 //     CTAs' "empty" and "TMEM full" barriers;
 //   * both CTAs' epilogues arrive on the leader's "TMEM empty" barrier.
+// Outlier columns (the 16-bit product): a kind::f16 MMA accumulates them into a
+// second (fp32) TMEM accumulator after the int8 K-blocks; TMEM then holds one
+// tile (int32 + fp32), otherwise two int32 accumulators are double-buffered.
 // No TMA load uses cluster multicast: each CTA loads its own halves.
 #include <cuda.h>
 
@@ -25,7 +28,7 @@ constexpr int BM = 128;           // rows per CTA (256 per pair)
 constexpr int BN = 256;           // output columns per tile
 constexpr int BN_HALF = BN / 2;   // B rows loaded per CTA
 constexpr int BKB = 128;          // bytes of K per stage
-constexpr int STAGES = 6;
+constexpr int STAGES = 5;
 constexpr int A_BYTES = BM * BKB;       // 16 KB
 constexpr int B_BYTES = BN_HALF * BKB;  // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -93,12 +96,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int num_m = static_cast<int>((p.T + 2 * BM - 1) / (2 * BM));
   const int num_n = static_cast<int>((p.N + BN - 1) / BN);
   const int num_tiles = num_m * num_n;
-  const int n_out = (p.n_out != nullptr) ? *p.n_out : 0;
-  const int nkb_o = (p.mode == 0) ? (n_out + 63) / 64 : 0;
-  const int nkb = p.nkb_i8 + nkb_o;
-  const bool has_out = nkb_o > 0;
-  const int nbuf = has_out ? 1 : 2;
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -115,10 +112,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (has_out) {
-      tma_prefetch_desc(&tmAo);
-      tma_prefetch_desc(&tmBo);
-    }
+    tma_prefetch_desc(&tmAo);
+    tma_prefetch_desc(&tmBo);
   }
   if (warp == 1) {
     tmem_alloc_pair(&tmem_base_sh, TMEM_COLS);
@@ -129,6 +124,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   cluster_sync();  // both CTAs' barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
+
+  // The set-up above overlaps the tail of the row quantisation (programmatic
+  // launch); n_out and every operand are read only after it has completed.
+  griddep_wait();
+  const int n_out = (p.n_out != nullptr && p.mode == 0) ? *p.n_out : 0;
+  const int nkb_o = (n_out + 63) / 64;
+  const int nkb = p.nkb_i8 + nkb_o;
+  const bool has_out = nkb_o > 0;                            // outliers on tensor cores (fp32 TMEM)
+  const int nbuf = has_out ? 1 : 2;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer (both CTAs)
@@ -235,36 +239,36 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t aph = static_cast<uint32_t>((it / nbuf) & 1);
       int m_blk, n_blk;
       tile_coords(tile, num_m, num_n, m_blk, n_blk);
-      if (!mbar_wait_cluster(&tfull_bar[buf], aph, &abort_sh, p.st, W_TFULL)) break;
-      tc_fence_after();
       const int64_t row = static_cast<int64_t>(m_blk) * 2 * BM + static_cast<int64_t>(rank) * BM + q * 32 + lane;
       const bool row_ok = row < p.T;
+      if (!mbar_wait_cluster(&tfull_bar[buf], aph, &abort_sh, p.st, W_TFULL)) break;
+      tc_fence_after();
       const float ra = (row_ok && p.mode == 0) ? __ldg(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
       #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        const int col0 = half * 128 + c * 32;
+      for (int c = 0; c < 8; ++c) {
+        const int col0 = half * 128 + c * 16;
         const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
-        uint32_t acc[32];
-        uint32_t fo[32];
-        tmem_ld_32x32b_x32(tmem_base + lane_base + static_cast<uint32_t>(buf) * 256u + col0, acc);
-        if (has_out) tmem_ld_32x32b_x32(tmem_base + lane_base + 256u + col0, fo);
+        uint32_t acc[16];
+        uint32_t fo[16];  // fp32 outlier product (when the tile has outlier columns)
+        tmem_ld_32x32b_x16(tmem_base + lane_base + static_cast<uint32_t>(buf) * 256u + col0, acc);
+        if (has_out) tmem_ld_32x32b_x16(tmem_base + lane_base + 256u + col0, fo);
         tmem_ld_wait();
         if (p.mode == 1) {
           if (row_ok) {
             int32_t* dst = p.acc_out + row * p.N + gcol0;
             #pragma unroll
-            for (int g = 0; g < 8; ++g)
+            for (int g = 0; g < 4; ++g)
               if (gcol0 + g * 4 + 4 <= p.N)
                 reinterpret_cast<int4*>(dst)[g] = make_int4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]);
           }
           continue;
         }
-        const int64_t my_col = gcol0 + lane;
+        const int64_t my_col = gcol0 + (lane & 15);
         const float scb_l = (my_col < p.N) ? __ldg(&p.SCB[my_col]) : 0.0f;
         const float b_l = (p.bias != nullptr && my_col < p.N) ? __half2float(p.bias[my_col]) : 0.0f;
-        uint32_t packed[16];
+        uint32_t packed[8];
         #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
+        for (int i = 0; i < 16; i += 2) {
           const float s0 = __shfl_sync(0xffffffffu, scb_l, i);
           const float s1 = __shfl_sync(0xffffffffu, scb_l, i + 1);
           const float b0 = __shfl_sync(0xffffffffu, b_l, i);
@@ -280,7 +284,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (row_ok) {
           __half* dst = p.Y + row * p.N + gcol0;
           #pragma unroll
-          for (int g = 0; g < 4; ++g)
+          for (int g = 0; g < 2; ++g)
             if (gcol0 + g * 8 + 8 <= p.N)
               reinterpret_cast<uint4*>(dst)[g] =
                   make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
@@ -396,17 +400,19 @@ cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s) {
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
 
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, gemm_i8_tc2_kernel, tmA, tmB, tmAo, tmBo, p);
 }
 

@@ -29,6 +29,7 @@ constexpr int DV_THREADS = DV_WARPS * 32;
 constexpr int DV_RG = 4;   // 8-row groups per pass (32 rows)
 constexpr int DV_U = 2;    // K-steps (64 B each) loaded before computing
 constexpr int DV_OB = 64;  // outlier columns staged per block
+constexpr int kPrefetchRows = 16;  // weight rows per CTA pulled into L2 before the wait
 
 struct DvParams {
   const int8_t* Xq;
@@ -77,6 +78,12 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
   const int64_t steps = (p.K + 63) / 64;
   const int64_t s_begin = steps * warp / DV_WARPS;
   const int64_t s_end = steps * (warp + 1) / DV_WARPS;
+  // The weights are an input of the layer, not an output of the preceding
+  // kernels: under a programmatic launch, start pulling this CTA's first rows
+  // into L2 while the outlier pass and the row quantisation finish.
+  if (threadIdx.x < kPrefetchRows && g_begin * 8 + threadIdx.x < g_end * 8)
+    prefetch_l2(p.CB + (g_begin * 8 + threadIdx.x) * p.K, static_cast<uint32_t>(p.K));
+  griddep_wait();
   const int n_out = (p.mode == 0) ? *p.n_out : 0;
   const bool row_a = g < p.T;
   const bool row_b = g + 8 < p.T;
@@ -217,8 +224,16 @@ cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s) {
   const int64_t groups = a.N / 8;
   int64_t grid = static_cast<int64_t>(num_sms) * 2;
   if (grid > groups) grid = groups;
-  gemv_i8_decode_kernel<<<static_cast<unsigned>(grid), DV_THREADS, 0, s>>>(p);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(DV_THREADS, 1, 1);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel, p);
 }
 
 }  // namespace i8mp
