@@ -118,12 +118,35 @@ i8_status int8_linear_forward_path(const void* X, int64_t T, int64_t K, const in
                                    cudaStream_t stream);
 
 /*
+ * The forward of a layer with has_fp16_weights=True (bitsandbytes
+ * Linear8bitLt docstring: the weights remain fp16 and are quantised on the fly
+ * during each forward pass).  Each call quantises W exactly as
+ * int8_quantize_weight does (into the workspace) and runs the forward; the
+ * outlier columns are multiplied with W's own fp16 columns W[:, idx] rather
+ * than the dequantised CB.
+ *   W         device fp16 [N,K]
+ *   workspace device, >= int8_linear_fp16w_workspace_bytes(T,K,N), 256-byte
+ *             aligned (the forward's workspace followed by CB [N,K], SCB [N]).
+ * Other arguments, results and errors as int8_linear_forward.
+ */
+size_t int8_linear_fp16w_workspace_bytes(int64_t T, int64_t K, int64_t N);
+i8_status int8_linear_forward_fp16w(const void* X, int64_t T, int64_t K, const void* W, const void* bias, int64_t N,
+                                    float threshold, void* Y, int32_t* idx, int32_t* n_out, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of
  * `workspace`: I8_OK, or I8_ERR_TIMEOUT if a kernel of the most recent
  * forward using this workspace gave up a wait.  *where (may be NULL)
- * receives the tag of the wait that gave up.
+ * receives the tag of the wait that gave up; 0xffffffff when the
+ * synchronisation itself failed (I8_ERR_CUDA, see int8_last_cuda_error), and
+ * 0xbad00000 | value when the status word holds a value no kernel writes.
  */
 i8_status int8_check_status(void* workspace, uint32_t* where, cudaStream_t stream);
+
+/* Text of the last CUDA error this thread's calls into the library met
+ * ("no error" if none).  Host-only. */
+const char* int8_last_cuda_error(void);
 
 /*
  * The forward with HOST activations and output: copies X host->device,
@@ -150,6 +173,32 @@ i8_status int8_linear_forward_timed(const void* X, int64_t T, int64_t K, const i
                                     const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
                                     int32_t* n_out, void* workspace, size_t workspace_bytes, int path,
                                     void* const* events, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Persistence of a quantised layer (host memory only; no CUDA call).
+ *
+ * The Hugging Face integration page lists, under "Future work and
+ * limitations", that INT8 checkpoints omitted the quantisation statistics
+ * CB/SCB, so a quantised layer could not be loaded directly.  These calls
+ * store CB, SCB and (optionally) the bias in one byte image and read them
+ * back, so a layer is loaded without its fp16 weight and without quantising
+ * again.  Image (little-endian): "I8MPLYR1", int64 N, int64 K, uint32 flags
+ * (bit 0 = bias present), uint32 0, then fp32 SCB[N], fp16 bias[N] if
+ * present, int8 CB[N*K] row-major.  Shapes follow the forward's rules.
+ * ------------------------------------------------------------------------- */
+
+/* Image size in bytes (0 for an unsupported shape). */
+size_t int8_layer_packed_bytes(int64_t N, int64_t K, int has_bias);
+/* Writes the image of host CB [N,K], SCB [N], bias [N] (or NULL) into `out`
+ * (>= int8_layer_packed_bytes bytes, else I8_ERR_WORKSPACE). */
+i8_status int8_layer_pack(const int8_t* CB, const float* SCB, const void* bias, int64_t N, int64_t K, void* out,
+                          size_t out_bytes);
+/* Validates an image (magic, shape rules, flags, length) and reads N, K and
+ * whether it holds a bias.  I8_ERR_INVALID_ARG for anything malformed. */
+i8_status int8_layer_unpack_header(const void* buf, size_t bytes, int64_t* N, int64_t* K, int* has_bias);
+/* Copies an image's SCB, bias (when present and `bias` is not NULL) and CB
+ * into host buffers sized from int8_layer_unpack_header. */
+i8_status int8_layer_unpack(const void* buf, size_t bytes, int8_t* CB, float* SCB, void* bias);
 
 /* ---------------------------------------------------------------------------
  * Inspection entry points (used by the parity tests; not needed for inference)

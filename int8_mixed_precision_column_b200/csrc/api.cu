@@ -99,7 +99,14 @@ uint32_t threshold_bits(float thr) {
   return lo;
 }
 
-inline i8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? I8_OK : I8_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// Maps a CUDA result to a status, remembering the error for int8_last_cuda_error().
+inline i8_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return I8_OK;
+  g_last_cuda_error = e;
+  return I8_ERR_CUDA;
+}
 
 // The product kernel: decode GEMV, or the tensor-core GEMM on SM pairs (the
 // single-SM GEMM when pairs are not launchable or when asked for explicitly).
@@ -111,7 +118,7 @@ cudaError_t launch_product(const GemmArgs& a, int path, bool gemv, int num_sms, 
 
 i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB, const void* bias,
                        int64_t N, float threshold, void* Y, int32_t* idx, int32_t* n_out, void* ws, size_t ws_bytes,
-                       int path, void* const* events, cudaStream_t stream) {
+                       int path, void* const* events, cudaStream_t stream, const __half* Wf = nullptr) {
   if (!shape_ok(T, K, N)) return I8_ERR_INVALID_ARG;
   if (path < kPathAuto || path > kPathTensorCoreSingleSM) return I8_ERR_INVALID_ARG;
   if (path == kPathDecode && T > kDecodeMaxT) return I8_ERR_INVALID_ARG;
@@ -161,8 +168,8 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   const bool gemv = (path == kPathDecode) || (path == kPathAuto && T <= kDecodeMaxT);
   // programmatic launches only directly after one of our kernels
   const bool after_outliers = (hb != 0xffffffffu);
-  e = launch_rowquant(Xh, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, num_sms, dst,
-                      after_outliers, stream);
+  e = launch_rowquant(Xh, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, Wf, num_sms,
+                      dst, after_outliers, stream);
   if (e != cudaSuccess || !mark(2)) return I8_ERR_CUDA;
 
   GemmArgs a;
@@ -184,6 +191,7 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   a.K = K;
   a.mode = 0;
   a.pdl = true;  // follows the row quantisation kernel
+  a.Wf = Wf;
   e = launch_product(a, path, gemv, num_sms, stream);
   if (e != cudaSuccess || !mark(3)) return I8_ERR_CUDA;
   return I8_OK;
@@ -259,13 +267,48 @@ i8_status int8_linear_forward_timed(const void* X, int64_t T, int64_t K, const i
 
 i8_status int8_check_status(void* workspace, uint32_t* where, cudaStream_t stream) {
   if (workspace == nullptr || !aligned(workspace, 256)) return I8_ERR_WORKSPACE;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return I8_ERR_CUDA;
+  if (where != nullptr) *where = 0xffffffffu;  // "the synchronisation itself failed"
+  i8_status st = cuda_status(cudaStreamSynchronize(stream));
+  if (st != I8_OK) return st;
   DevStatus h;
-  if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return I8_ERR_CUDA;
+  st = cuda_status(cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost));
+  if (st != I8_OK) return st;
   if (where != nullptr) *where = h.where;
   if (h.error == 0) return I8_OK;
-  if (cudaMemset(workspace, 0, 2 * sizeof(uint32_t)) != cudaSuccess) return I8_ERR_CUDA;
-  return h.error == kErrTimeout ? I8_ERR_TIMEOUT : I8_ERR_CUDA;
+  st = cuda_status(cudaMemset(workspace, 0, 2 * sizeof(uint32_t)));
+  if (st != I8_OK) return st;
+  if (h.error == kErrTimeout) return I8_ERR_TIMEOUT;
+  if (where != nullptr) *where = 0xbad00000u | (h.error & 0xfffffu);  // not a code the kernels write
+  return I8_ERR_CUDA;
+}
+
+const char* int8_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+
+// has_fp16_weights=True: the forward's workspace, then CB [N,K] and SCB [N].
+size_t int8_linear_fp16w_workspace_bytes(int64_t T, int64_t K, int64_t N) {
+  if (!shape_ok(T, K, N)) return 0;
+  const int8_ws_layout L = make_layout(T, K, N);
+  return static_cast<size_t>(align_up(align_up(L.total + static_cast<uint64_t>(N) * K, 256) + N * 4, 256));
+}
+
+i8_status int8_linear_forward_fp16w(const void* X, int64_t T, int64_t K, const void* W, const void* bias, int64_t N,
+                                    float threshold, void* Y, int32_t* idx, int32_t* n_out, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
+  if (!shape_ok(T, K, N)) return I8_ERR_INVALID_ARG;
+  if (W == nullptr || !aligned(W, 16)) return I8_ERR_INVALID_ARG;
+  const int8_ws_layout L = make_layout(T, K, N);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < int8_linear_fp16w_workspace_bytes(T, K, N))
+    return I8_ERR_WORKSPACE;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  int8_t* CB = reinterpret_cast<int8_t*>(w + L.total);
+  float* SCB = reinterpret_cast<float*>(w + align_up(L.total + static_cast<uint64_t>(N) * K, 256));
+  int num_sms = 0;
+  i8_status st = device_info(&num_sms);
+  if (st != I8_OK) return st;
+  // the weight is quantised anew in every forward (Linear8bitLt, has_fp16_weights=True)
+  if (launch_quantize_weight(static_cast<const __half*>(W), N, K, CB, SCB, stream) != cudaSuccess) return I8_ERR_CUDA;
+  return forward_impl(X, T, K, CB, SCB, bias, N, threshold, Y, idx, n_out, workspace, L.total, 0, nullptr, stream,
+                      static_cast<const __half*>(W));
 }
 
 size_t int8_linear_forward_host_workspace_bytes(int64_t T, int64_t K, int64_t N) {

@@ -55,6 +55,8 @@ struct Params {
   const int32_t* n_out;
   DevStatus* st;
   int mode;
+  int vec_scb;   // SCB is 16-byte aligned: a tile's 16 column scales load as 4 x float4
+  int vec_bias;  // bias is 16-byte aligned: 16 halves load as 2 x uint4
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
@@ -263,18 +265,49 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           continue;
         }
-        const int64_t my_col = gcol0 + (lane & 15);
-        const float scb_l = (my_col < p.N) ? __ldg(&p.SCB[my_col]) : 0.0f;
-        const float b_l = (p.bias != nullptr && my_col < p.N) ? __half2float(p.bias[my_col]) : 0.0f;
+        // column scales and bias of these 16 columns: every lane reads the same
+        // addresses, so the loads are L1 broadcasts
+        float sc[16], bi[16];
+        const bool full = gcol0 + 16 <= p.N;
+        if (full && p.vec_scb) {
+          const float4* s4 = reinterpret_cast<const float4*>(p.SCB + gcol0);
+          #pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 v = __ldg(s4 + q4);
+            sc[4 * q4] = v.x;
+            sc[4 * q4 + 1] = v.y;
+            sc[4 * q4 + 2] = v.z;
+            sc[4 * q4 + 3] = v.w;
+          }
+        } else {
+          #pragma unroll
+          for (int i = 0; i < 16; ++i) sc[i] = (gcol0 + i < p.N) ? __ldg(&p.SCB[gcol0 + i]) : 0.0f;
+        }
+        if (p.bias == nullptr) {
+          #pragma unroll
+          for (int i = 0; i < 16; ++i) bi[i] = 0.0f;
+        } else if (full && p.vec_bias) {
+          const uint4* b8 = reinterpret_cast<const uint4*>(p.bias + gcol0);
+          #pragma unroll
+          for (int q8 = 0; q8 < 2; ++q8) {
+            const uint4 v = __ldg(b8 + q8);
+            const __half2* h = reinterpret_cast<const __half2*>(&v);
+            #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(h[e]);
+              bi[8 * q8 + 2 * e] = f.x;
+              bi[8 * q8 + 2 * e + 1] = f.y;
+            }
+          }
+        } else {
+          #pragma unroll
+          for (int i = 0; i < 16; ++i) bi[i] = (gcol0 + i < p.N) ? __half2float(p.bias[gcol0 + i]) : 0.0f;
+        }
         uint32_t packed[8];
         #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          const float s0 = __shfl_sync(0xffffffffu, scb_l, i);
-          const float s1 = __shfl_sync(0xffffffffu, scb_l, i + 1);
-          const float b0 = __shfl_sync(0xffffffffu, b_l, i);
-          const float b1 = __shfl_sync(0xffffffffu, b_l, i + 1);
-          float y0 = static_cast<float>(static_cast<int32_t>(acc[i])) * (ra * s0) + b0;
-          float y1 = static_cast<float>(static_cast<int32_t>(acc[i + 1])) * (ra * s1) + b1;
+          float y0 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i])), ra * sc[i], bi[i]);
+          float y1 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i + 1])), ra * sc[i + 1], bi[i + 1]);
           if (has_out) {
             y0 += __uint_as_float(fo[i]);
             y1 += __uint_as_float(fo[i + 1]);
@@ -395,6 +428,8 @@ cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s) {
   p.n_out = outl ? a.n_out : nullptr;
   p.st = a.st;
   p.mode = a.mode;
+  p.vec_scb = (reinterpret_cast<uintptr_t>(a.SCB) % 16 == 0) ? 1 : 0;
+  p.vec_bias = (a.bias != nullptr && reinterpret_cast<uintptr_t>(a.bias) % 16 == 0) ? 1 : 0;
   const int64_t tiles = ((a.T + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
   if (tiles > 0x3fffffff) return cudaErrorInvalidValue;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);

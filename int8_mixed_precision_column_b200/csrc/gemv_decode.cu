@@ -41,6 +41,7 @@ struct DvParams {
   int64_t ldo;
   const int32_t* idx;
   const int32_t* n_out;
+  const __half* Wf;  // fp16 weight (has_fp16_weights=True) or null
   __half* Y;
   int32_t* acc_out;
   int64_t T, N, K;
@@ -164,8 +165,13 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
         const int64_t j = g0 * 8 + r;
         float wv = 0.0f;
         if (j < g_end * 8) {
-          const float cbv = static_cast<float>(__ldg(&p.CB[j * p.K + __ldg(&p.idx[ob + o])]));
-          wv = __half2float(__float2half_rn(__fdiv_rn(__fmul_rn(cbv, __ldg(&p.SCB[j])), 127.0f)));
+          const int64_t col = __ldg(&p.idx[ob + o]);
+          if (p.Wf != nullptr) {
+            wv = __half2float(p.Wf[j * p.K + col]);
+          } else {
+            const float cbv = static_cast<float>(__ldg(&p.CB[j * p.K + col]));
+            wv = __half2float(__float2half_rn(__fdiv_rn(__fmul_rn(cbv, __ldg(&p.SCB[j])), 127.0f)));
+          }
         }
         wo_s[r][o] = wv;
       }
@@ -215,6 +221,7 @@ cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s) {
   p.ldo = a.ldo;
   p.idx = a.idx;
   p.n_out = a.n_out;
+  p.Wf = a.Wf;
   p.Y = a.Y;
   p.acc_out = a.acc_out;
   p.T = a.T;

@@ -21,15 +21,16 @@ cudaError_t launch_quantize_weight(const __half* W, int64_t N, int64_t K, int8_t
 cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
                             uint32_t* prefix, int32_t* idx, int32_t* n_out, DevStatus* st, cudaStream_t s);
 
-// `pdl`: launch with programmatic stream serialisation (only when the previous
-// operation in the stream is the outlier-pass kernel).
 // Row-wise absmax int8 quantisation over non-outlier columns, fp16 gather of
 // the outlier activation columns into Xo, and (when `with_wo`) the gather and
-// dequantisation of the matching weight columns into Wo.
+// dequantisation of the matching weight columns into Wo -- or, when `Wf` (the
+// fp16 weight of a has_fp16_weights=True layer) is given, its own columns.
+// `pdl`: launch with programmatic stream serialisation (only when the previous
+// operation in the stream is the outlier-pass kernel).
 cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_t* mask, const uint32_t* prefix,
                             const int32_t* idx, const int32_t* n_out, int8_t* Xq, float* sA, __half* Xo,
                             int64_t ldo, const int8_t* CB, const float* SCB, int64_t N, __half* Wo, bool with_wo,
-                            int num_sms, DevStatus* st, bool pdl, cudaStream_t s);
+                            const __half* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s);
 
 struct GemmArgs {
   const int8_t* Xq;      // [T,K]
@@ -48,6 +49,7 @@ struct GemmArgs {
   int64_t T, N, K;
   int mode;              // 0: fused fp16 Y, 1: int32 accumulators only
   bool pdl = false;      // launch with programmatic stream serialisation (previous op is our kernel)
+  const __half* Wf = nullptr;  // fp16 weight [N,K] (has_fp16_weights=True): outlier weights come from it
 };
 
 // Prefill: persistent tcgen05 kind::i8 GEMM with TMEM accumulators, fused

@@ -114,7 +114,7 @@ extern "C" i8_status int8_linear_forward_decode_static(const void* X, int64_t T,
     e = launch_outliers(Xh, T, K, hb, mask, mask + (K + 31) / 32, idx, n_out, dst, stream);
   if (e != cudaSuccess) return I8_ERR_CUDA;
   e = launch_rowquant(Xh, T, K, mask, mask + (K + 31) / 32, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, nullptr,
-                      false, num_sms, dst, hb != 0xffffffffu, stream);
+                      false, nullptr, num_sms, dst, hb != 0xffffffffu, stream);
   if (e != cudaSuccess) return I8_ERR_CUDA;
 
   GemmArgs a;

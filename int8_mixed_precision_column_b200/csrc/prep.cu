@@ -65,19 +65,31 @@ cudaError_t launch_quantize_weight(const __half* W, int64_t N, int64_t K, int8_t
 // <= threshold (computed on the host).  NaN patterns (> 0x7c00) are excluded so
 // that NaN never flags a column.
 // CTA shape: `wc` of the 8 warps sit side by side along the columns (each warp
-// 256 columns = 512 contiguous bytes of a row), the other 8/wc split the rows.
-// Large T uses wc = 8 (a CTA reads 4 KB contiguous of each of its rows, 8 rows
-// of loads in flight per thread); small T uses wc = 1 so that enough CTAs
-// exist.  Four lanes' flag bytes make one mask word, ORed into the mask with
-// one atomicOr.  The last CTA to finish compacts the mask into the ascending
+// 256 columns = 512 contiguous bytes of a row), the other 8/wc split the rows;
+// the launcher uses wc = 1.  Four lanes' flag bytes make one mask word, ORed
+// into the mask with one atomicOr.  The last CTA to finish compacts the mask into the ascending
 // idx list and records, per mask word, how many outlier columns precede it
 // (prefix), so that the rank of an outlier column is prefix[w] + popc(lower
 // bits of word w).
 // ---------------------------------------------------------------------------
 constexpr int kMaskThreads = 256;
-constexpr int kMaskUnroll = 8;
+constexpr int kMaskUnroll = 4;
 
+// Largest magnitude bit pattern among the 8 halves of v (fp16 max of |x|; max
+// ignores a NaN operand, so a NaN can only raise the result to a NaN pattern
+// when every element is NaN -- the caller then takes the exact path).
+__device__ __forceinline__ uint32_t chunk_max_mag(const uint4& v) {
+  const uint32_t w[4] = {v.x & 0x7fff7fffu, v.y & 0x7fff7fffu, v.z & 0x7fff7fffu, v.w & 0x7fff7fffu};
+  const __half2 m = __hmax2(__hmax2(*reinterpret_cast<const __half2*>(&w[0]), *reinterpret_cast<const __half2*>(&w[1])),
+                            __hmax2(*reinterpret_cast<const __half2*>(&w[2]), *reinterpret_cast<const __half2*>(&w[3])));
+  const uint32_t mm = *reinterpret_cast<const uint32_t*>(&m);
+  return max(mm & 0xffffu, mm >> 16);
+}
+
+// Exact flags of one 8-column chunk; chunks whose largest magnitude is not
+// above the threshold (nearly all of them) are settled by chunk_max_mag alone.
 __device__ __forceinline__ uint32_t flag_bits8(const uint4& v, uint32_t h2) {
+  if (chunk_max_mag(v) <= (h2 & 0xffffu)) return 0u;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t bits = 0;
   #pragma unroll
@@ -172,9 +184,10 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const __half
 
 cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
                             uint32_t* prefix, int32_t* idx, int32_t* n_out, DevStatus* st, cudaStream_t s) {
-  // Large T: 8 warps along the columns, 64-row chunks.  Small T: warps split the rows.
-  const int wc = (T >= 512) ? 8 : 1;
-  const int64_t rows_per_cta = (wc == 8) ? 64 : 128;
+  // The 8 warps split the rows (measured faster than warps side by side along
+  // the columns, which gives fewer, longer-lived CTAs).
+  const int wc = 1;
+  const int64_t rows_per_cta = 128;
   const int64_t slabs = (K + 256 * wc - 1) / (256 * wc);
   const int64_t chunks = (T + rows_per_cta - 1) / rows_per_cta;
   if (slabs > 0x7fffffff || chunks > 65535) return cudaErrorInvalidValue;
@@ -186,40 +199,60 @@ cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbit
 // ---------------------------------------------------------------------------
 // Row quantisation + outlier gathers.
 //
-// Blocks [0, T): one CTA per token row t.  The row is read once into registers
-// (8 columns per 16-byte chunk), the absmax over non-outlier columns is
-// reduced across the CTA, and the codes are written as 8-byte packets.  Each
-// outlier value goes from registers straight to Xo[t, rank], its rank among
-// the outlier columns being prefix[word] + popc(lower bits of the word); Xo is
-// zero-padded to the next multiple of 64 (the K-block of the fp16 outlier MMA).
-// Blocks [T, ...): Wo[j, o] = fp16((CB[j, idx[o]] * SCB[j]) / 127) with the
-// same padding (only when the tensor-core path consumes Wo), four independent
-// gathers per thread in flight.
+// Rows: one warp per token row t, two passes over the row (the second mostly
+// from L1/L2), with 8 independent 16-byte loads in flight per lane.
+//   pass 1: absmax over the non-outlier columns, kept as an fp16 magnitude bit
+//           pattern (integer max of (bits & 0x7fff) equals the magnitude max
+//           for finite values); chunks without outlier columns use an fp16 max
+//           of |x|; a warp shuffle reduces it -- no block barrier;
+//   pass 2: codes clamp(round_half_away(x * fp32(127/absmax))) packed 8 per
+//           8-byte store, outlier values written to Xo[t, rank] straight from
+//           registers, rank = prefix[word] + popc(lower bits of the word).
+// Xo is zero-padded to the next multiple of 64 (the fp16 outlier K-block).
+// Wo blocks (blockIdx >= row blocks): Wo[j, o] = fp16((CB[j, idx[o]] * SCB[j]) / 127)
+// with the same padding, four independent gathers per thread in flight (only
+// when the tensor-core product consumes Wo).
 // ---------------------------------------------------------------------------
 constexpr int kRowThreads = 256;
-constexpr int kRowChunks = 8;   // registers hold rows up to 256*8*8 = 16384 columns
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kRowUnroll = 8;
 constexpr int kWoUnroll = 4;
 
 __device__ __forceinline__ uint32_t mask_byte(const uint32_t* mask, int64_t chunk) {
   return (__ldg(&mask[chunk >> 2]) >> ((chunk & 3) * 8)) & 0xffu;
 }
 
-__device__ __forceinline__ float row_absmax_part(const uint4& v, uint32_t mb) {
-  const __half* h = reinterpret_cast<const __half*>(&v);
-  float m = 0.0f;
+// Largest magnitude pattern among the non-outlier elements of a chunk.
+__device__ __forceinline__ uint32_t chunk_max_mag_kept(const uint4& v, uint32_t mb) {
+  if (mb == 0) return chunk_max_mag(v);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
   #pragma unroll
   for (int e = 0; e < 8; ++e)
-    if (!((mb >> e) & 1u)) m = fmaxf(m, fabsf(__half2float(h[e])));
+    if (!((mb >> e) & 1u)) m = max(m, (w[e >> 1] >> ((e & 1) * 16)) & 0x7fffu);
   return m;
 }
 
-__device__ __forceinline__ uint2 row_codes(const uint4& v, uint32_t mb, float inv) {
-  const __half* h = reinterpret_cast<const __half*>(&v);
+// Round half away from zero for |y| <= 127 * (1 + 2^-23), the range of
+// x * fp32(127/absmax) when |x| <= absmax.  For |y| >= 0.5, |y| + 0.5 is either
+// exact or rounds within the same integer interval, so truncating it gives
+// the nearest integer with ties away from zero; |y| < 0.5 gives 0.
+__device__ __forceinline__ int round_away_code(float y) {
+  const float a = fabsf(y);
+  int q = (a < 0.5f) ? 0 : __float2int_rz(a + 0.5f);
+  q = min(q, 127);
+  return (y < 0.0f) ? -q : q;
+}
+
+__device__ __forceinline__ uint2 row_codes_fast(const uint4& v, uint32_t mb, float inv) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
   uint32_t w[2] = {0u, 0u};
   #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int q = ((mb >> e) & 1u) ? 0 : quant_code(__half2float(h[e]), inv);
-    w[e >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (e & 3));
+  for (int p = 0; p < 4; ++p) {
+    const float2 f = __half22float2(h[p]);
+    const int q0 = ((mb >> (2 * p)) & 1u) ? 0 : round_away_code(__fmul_rn(f.x, inv));
+    const int q1 = ((mb >> (2 * p + 1)) & 1u) ? 0 : round_away_code(__fmul_rn(f.y, inv));
+    w[p >> 1] |= ((static_cast<uint32_t>(q0) & 0xffu) | ((static_cast<uint32_t>(q1) & 0xffu) << 8)) << (16 * (p & 1));
   }
   return make_uint2(w[0], w[1]);
 }
@@ -236,41 +269,43 @@ __device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, in
     if ((mb >> e) & 1u) xo_row[base + __popc(mw & ((1u << (sh + e)) - 1u))] = h[e];
 }
 
-__global__ void __launch_bounds__(kRowThreads, 3) rowquant_regs_kernel(
+__global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
     const __half* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
     const uint32_t* __restrict__ prefix, const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p,
     int8_t* __restrict__ Xq, float* __restrict__ sA, __half* __restrict__ Xo, int64_t ldo,
     const int8_t* __restrict__ CB, const float* __restrict__ SCB, int64_t N, __half* __restrict__ Wo,
-    int64_t wo_blocks) {
-  __shared__ float s_red[kRowThreads / 32];
-  const int tid = threadIdx.x;
+    const __half* __restrict__ Wf, int64_t row_blocks, int64_t wo_blocks) {
+  const int lane = threadIdx.x & 31;
   griddep_launch_dependents();
   griddep_wait();  // mask, prefix, idx, n_out come from the outlier pass
   const int n_out = *n_out_p;
   const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
 
-  if (static_cast<int64_t>(blockIdx.x) >= T) {
+  if (static_cast<int64_t>(blockIdx.x) >= row_blocks) {
     // ---- Wo rows ----
     if (n_out == 0) return;
     const int64_t total = N * npad;
     const int64_t stride = wo_blocks * kRowThreads * kWoUnroll;
-    for (int64_t e0 = (static_cast<int64_t>(blockIdx.x) - T) * kRowThreads * kWoUnroll + tid; e0 < total;
-         e0 += stride) {
+    for (int64_t e0 = (static_cast<int64_t>(blockIdx.x) - row_blocks) * kRowThreads * kWoUnroll + threadIdx.x;
+         e0 < total; e0 += stride) {
       int8_t cbv[kWoUnroll];
+      __half wfv[kWoUnroll];
       int64_t jj[kWoUnroll], oo[kWoUnroll];
       #pragma unroll
       for (int u = 0; u < kWoUnroll; ++u) {
         const int64_t e = e0 + static_cast<int64_t>(u) * kRowThreads;
         jj[u] = e / npad;
         oo[u] = e - jj[u] * npad;
-        cbv[u] = (e < total && oo[u] < n_out) ? __ldg(&CB[jj[u] * K + __ldg(&idx[oo[u]])]) : int8_t(0);
+        const bool live = e < total && oo[u] < n_out;
+        cbv[u] = (live && Wf == nullptr) ? __ldg(&CB[jj[u] * K + __ldg(&idx[oo[u]])]) : int8_t(0);
+        wfv[u] = (live && Wf != nullptr) ? Wf[jj[u] * K + __ldg(&idx[oo[u]])] : __float2half_rn(0.0f);
       }
       #pragma unroll
       for (int u = 0; u < kWoUnroll; ++u) {
         const int64_t e = e0 + static_cast<int64_t>(u) * kRowThreads;
         if (e < total) {
-          __half v = __float2half_rn(0.0f);
-          if (oo[u] < n_out)
+          __half v = wfv[u];
+          if (oo[u] < n_out && Wf == nullptr)
             v = __float2half_rn(__fdiv_rn(__fmul_rn(static_cast<float>(cbv[u]), __ldg(&SCB[jj[u]])), 127.0f));
           Wo[jj[u] * ldo + oo[u]] = v;
         }
@@ -279,197 +314,58 @@ __global__ void __launch_bounds__(kRowThreads, 3) rowquant_regs_kernel(
     return;
   }
 
-  // ---- one token row ----
-  const int64_t t = blockIdx.x;
+  // ---- one warp per token row ----
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
   const int64_t nv = K / 8;
   const uint4* src = reinterpret_cast<const uint4*>(X + t * K);
-  uint4 v[kRowChunks];
-  uint32_t mb[kRowChunks];
-  float m = 0.0f;
-  #pragma unroll
-  for (int c = 0; c < kRowChunks; ++c) {
-    const int64_t i = tid + static_cast<int64_t>(c) * kRowThreads;
-    if (i < nv) {
-      v[c] = __ldcs(src + i);
-      mb[c] = mask_byte(mask, i);
-      m = fmaxf(m, row_absmax_part(v[c], mb[c]));
+  uint32_t mmax = 0;
+  for (int64_t c0 = lane; c0 < nv; c0 += 32 * kRowUnroll) {
+    uint4 v[kRowUnroll];
+    #pragma unroll
+    for (int u = 0; u < kRowUnroll; ++u) {
+      const int64_t c = c0 + 32 * u;
+      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+    #pragma unroll
+    for (int u = 0; u < kRowUnroll; ++u) {
+      const int64_t c = c0 + 32 * u;
+      if (c < nv) mmax = max(mmax, chunk_max_mag_kept(v[u], mask_byte(mask, c)));
     }
   }
-  for (int64_t i = tid + static_cast<int64_t>(kRowChunks) * kRowThreads; i < nv; i += kRowThreads)
-    m = fmaxf(m, row_absmax_part(__ldg(src + i), mask_byte(mask, i)));
-  m = warp_max(m);
-  if ((tid & 31) == 0) s_red[tid >> 5] = m;
-  __syncthreads();
-  if (tid < 32) {
-    float r = (tid < kRowThreads / 32) ? s_red[tid] : 0.0f;
-    r = warp_max(r);
-    if (tid == 0) s_red[0] = r;
-  }
-  __syncthreads();
-  const float absmax = s_red[0];
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+  const float absmax = __half2float(__ushort_as_half(static_cast<unsigned short>(mmax)));
   const float inv = scale_inv(absmax);
-  if (tid == 0) sA[t] = absmax;
+  if (lane == 0) sA[t] = absmax;
+
   uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
   __half* xo_row = Xo + t * ldo;
-  #pragma unroll
-  for (int c = 0; c < kRowChunks; ++c) {
-    const int64_t i = tid + static_cast<int64_t>(c) * kRowThreads;
-    if (i < nv) {
-      dst[i] = row_codes(v[c], mb[c], inv);
-      if (mb[c]) scatter_outliers(v[c], mb[c], i, mask, prefix, xo_row);
-    }
-  }
-  for (int64_t i = tid + static_cast<int64_t>(kRowChunks) * kRowThreads; i < nv; i += kRowThreads) {
-    const uint4 vv = __ldg(src + i);
-    const uint32_t b = mask_byte(mask, i);
-    dst[i] = row_codes(vv, b, inv);
-    if (b) scatter_outliers(vv, b, i, mask, prefix, xo_row);
-  }
-  for (int64_t o = n_out + tid; o < npad; o += kRowThreads) xo_row[o] = __float2half_rn(0.0f);
-}
-
-// Bulk-copy variant for K <= kBulkMaxK: CTA b walks rows b, b+G, b+2G, ... with
-// two shared-memory stages.  One 1-D bulk copy brings a whole fp16 row in,
-// the codes are written to shared memory and leave with one bulk store, while
-// the next row's copy is already in flight.  One thread waits on each load's
-// mbarrier (bounded), the CTA barrier publishes it to the others.  After its
-// rows, each CTA takes a 1/G share of the Wo gather (when asked for).
-constexpr int64_t kBulkMaxK = 16384;
-constexpr uint32_t W_ROWLOAD = 0x301;
-
-__device__ __forceinline__ void wo_gather_share(const int8_t* __restrict__ CB, const float* __restrict__ SCB,
-                                                const int32_t* __restrict__ idx, int n_out, int64_t npad, int64_t N,
-                                                int64_t K, __half* __restrict__ Wo, int64_t ldo, int64_t part,
-                                                int64_t parts) {
-  const int64_t total = N * npad;
-  const int64_t stride = parts * kRowThreads * kWoUnroll;
-  for (int64_t e0 = part * kRowThreads * kWoUnroll + threadIdx.x; e0 < total; e0 += stride) {
-    int8_t cbv[kWoUnroll];
-    int64_t jj[kWoUnroll], oo[kWoUnroll];
+  for (int64_t c0 = lane; c0 < nv; c0 += 32 * kRowUnroll) {
+    uint4 v[kRowUnroll];
     #pragma unroll
-    for (int u = 0; u < kWoUnroll; ++u) {
-      const int64_t e = e0 + static_cast<int64_t>(u) * kRowThreads;
-      jj[u] = e / npad;
-      oo[u] = e - jj[u] * npad;
-      cbv[u] = (e < total && oo[u] < n_out) ? __ldg(&CB[jj[u] * K + __ldg(&idx[oo[u]])]) : int8_t(0);
+    for (int u = 0; u < kRowUnroll; ++u) {
+      const int64_t c = c0 + 32 * u;
+      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
     }
     #pragma unroll
-    for (int u = 0; u < kWoUnroll; ++u) {
-      const int64_t e = e0 + static_cast<int64_t>(u) * kRowThreads;
-      if (e < total) {
-        __half v = __float2half_rn(0.0f);
-        if (oo[u] < n_out)
-          v = __float2half_rn(__fdiv_rn(__fmul_rn(static_cast<float>(cbv[u]), __ldg(&SCB[jj[u]])), 127.0f));
-        Wo[jj[u] * ldo + oo[u]] = v;
+    for (int u = 0; u < kRowUnroll; ++u) {
+      const int64_t c = c0 + 32 * u;
+      if (c < nv) {
+        const uint32_t mb = mask_byte(mask, c);
+        dst[c] = row_codes_fast(v[u], mb, inv);
+        if (mb) scatter_outliers(v[u], mb, c, mask, prefix, xo_row);
       }
     }
   }
-}
-
-__global__ void __launch_bounds__(kRowThreads) rowquant_bulk_kernel(
-    const __half* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
-    const uint32_t* __restrict__ prefix, const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p,
-    int8_t* __restrict__ Xq, float* __restrict__ sA, __half* __restrict__ Xo, int64_t ldo,
-    const int8_t* __restrict__ CB, const float* __restrict__ SCB, int64_t N, __half* __restrict__ Wo, int with_wo,
-    DevStatus* st) {
-  extern __shared__ __align__(128) uint8_t rq_smem[];
-  __shared__ __align__(8) uint64_t bar[2];
-  __shared__ float s_red[kRowThreads / 32];
-  __shared__ volatile int s_abort;
-  const int tid = threadIdx.x;
-  const int64_t G = gridDim.x;
-  griddep_launch_dependents();
-
-  __half* xs[2] = {reinterpret_cast<__half*>(rq_smem), reinterpret_cast<__half*>(rq_smem + 2 * K)};
-  int8_t* qs[2] = {reinterpret_cast<int8_t*>(rq_smem + 4 * K), reinterpret_cast<int8_t*>(rq_smem + 5 * K)};
-  const uint32_t row_bytes = static_cast<uint32_t>(2 * K);
-  const int64_t nv = K / 8;
-  if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    s_abort = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-  if (tid == 0) {
-    // X is an input of the forward, not an output of the outlier pass: its
-    // first two rows can stream in before that pass has finished.
-    for (int b = 0; b < 2; ++b) {
-      const int64_t r = blockIdx.x + b * G;
-      if (r < T) {
-        mbar_arrive_expect_tx(&bar[b], row_bytes);
-        bulk_load(xs[b], X + r * K, row_bytes, &bar[b]);
-      }
-    }
-  }
-  griddep_wait();  // mask, prefix, idx, n_out come from the outlier pass
-  const int n_out = *n_out_p;
-  const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
-  int i = 0;
-  for (int64_t t = blockIdx.x; t < T; t += G, ++i) {
-    const int buf = i & 1;
-    if (tid == 0) mbar_wait(&bar[buf], static_cast<uint32_t>((i >> 1) & 1), &s_abort, st, W_ROWLOAD);
-    __syncthreads();
-    if (s_abort) break;
-    const __half* xrow = xs[buf];
-    float m = 0.0f;
-    for (int64_t c = tid; c < nv; c += kRowThreads)
-      m = fmaxf(m, row_absmax_part(reinterpret_cast<const uint4*>(xrow)[c], mask_byte(mask, c)));
-    m = warp_max(m);
-    if ((tid & 31) == 0) s_red[tid >> 5] = m;
-    if (tid == 0 && i >= 2) bulk_wait_read<1>();  // the store that last used qs[buf] has read it
-    __syncthreads();
-    float absmax = (tid < kRowThreads / 32) ? s_red[tid] : 0.0f;
-    absmax = warp_max(absmax);  // warp 0 holds the block maximum in every lane
-    __syncthreads();
-    if (tid == 0) s_red[0] = absmax;
-    __syncthreads();
-    absmax = s_red[0];
-    const float inv = scale_inv(absmax);
-    __half* xo_row = Xo + t * ldo;
-    for (int64_t c = tid; c < nv; c += kRowThreads) {
-      const uint4 v = reinterpret_cast<const uint4*>(xrow)[c];
-      const uint32_t mb = mask_byte(mask, c);
-      reinterpret_cast<uint2*>(qs[buf])[c] = row_codes(v, mb, inv);
-      if (mb) scatter_outliers(v, mb, c, mask, prefix, xo_row);
-    }
-    for (int64_t o = n_out + tid; o < npad; o += kRowThreads) xo_row[o] = __float2half_rn(0.0f);
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      sA[t] = absmax;
-      bulk_store(Xq + t * K, qs[buf], static_cast<uint32_t>(K));
-      bulk_commit();
-      const int64_t rn = t + 2 * G;
-      if (rn < T) {
-        mbar_arrive_expect_tx(&bar[buf], row_bytes);
-        bulk_load(xs[buf], X + rn * K, row_bytes, &bar[buf]);
-      }
-    }
-  }
-  if (tid == 0) {
-    bulk_wait<0>();
-    // loads still in flight after an early exit must land before the CTA ends
-    if (s_abort) {
-      volatile int never = 0;
-      for (int b = 0; b < 2; ++b) mbar_wait(&bar[b], static_cast<uint32_t>(((i + b) >> 1) & 1), &never, st, W_ROWLOAD);
-    }
-  }
-  if (with_wo && n_out > 0 && !s_abort) wo_gather_share(CB, SCB, idx, n_out, npad, N, K, Wo, ldo, blockIdx.x, G);
+  for (int64_t o = n_out + lane; o < npad; o += 32) xo_row[o] = __float2half_rn(0.0f);
 }
 
 cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_t* mask, const uint32_t* prefix,
                             const int32_t* idx, const int32_t* n_out, int8_t* Xq, float* sA, __half* Xo, int64_t ldo,
-                            const int8_t* CB, const float* SCB, int64_t N, __half* Wo, bool with_wo, int num_sms,
-                            DevStatus* st, bool pdl, cudaStream_t s) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kRowThreads, 1, 1);
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+                            const int8_t* CB, const float* SCB, int64_t N, __half* Wo, bool with_wo,
+                            const __half* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s) {
+  (void)st;
   int64_t wo_blocks = 0;
   if (with_wo) {
     wo_blocks = (N * 64 + kRowThreads * kWoUnroll - 1) / (kRowThreads * kWoUnroll);
@@ -477,35 +373,21 @@ cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_
     if (wo_blocks > cap) wo_blocks = cap;
     if (wo_blocks < 1) wo_blocks = 1;
   }
-  if (K <= kBulkMaxK) {
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 64 && !attr_done[dev]) {
-      e = cudaFuncSetAttribute(rowquant_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(6 * kBulkMaxK));
-      if (e != cudaSuccess) return e;
-      attr_done[dev] = true;
-    }
-    // two CTAs per SM (two staged rows each); enough CTAs for the rows, and for
-    // the Wo gather when the tensor-core product needs Wo
-    int64_t ctas = T;
-    if (with_wo && ctas < 2 * num_sms) ctas = 2 * num_sms;
-    if (ctas > 2 * num_sms) ctas = 2 * num_sms;
-    if (ctas == 0) return cudaSuccess;
-    cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(6 * K);
-    return cudaLaunchKernelEx(&cfg, rowquant_bulk_kernel, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB,
-                              N, Wo, with_wo ? 1 : 0, st);
-  }
-  const int64_t blocks = T + wo_blocks;
+  const int64_t row_blocks = (T + kRowWarps - 1) / kRowWarps;
+  const int64_t blocks = row_blocks + wo_blocks;
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&cfg, rowquant_regs_kernel, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N,
-                            Wo, wo_blocks);
+  cfg.blockDim = dim3(kRowThreads, 1, 1);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, rowquant_kernel, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N, Wo,
+                            Wf, row_blocks, wo_blocks);
 }
 
 }  // namespace i8mp

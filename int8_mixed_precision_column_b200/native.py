@@ -59,6 +59,14 @@ SIGNATURES = {
     "int8_gemm_i32": (_I32, [_P, _I64, _I64, _P, _I64, _P, _I32, _P, _SZ, _P]),
     "int8_outlier_threshold_bits": (ctypes.c_uint32, [_F32]),
     "int8_selftest_wait_timeout": (_I32, [_P, _SZ, ctypes.c_uint32, _P]),
+    "int8_linear_fp16w_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "int8_linear_forward_fp16w": (_I32, [_P, _I64, _I64, _P, _P, _I64, _F32, _P, _P, _P, _P, _SZ, _P]),
+    "int8_last_cuda_error": (ctypes.c_char_p, []),
+    "int8_layer_packed_bytes": (_SZ, [_I64, _I64, _I32]),
+    "int8_layer_pack": (_I32, [_P, _P, _P, _I64, _I64, _P, _SZ]),
+    "int8_layer_unpack_header": (_I32, [_P, _SZ, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                                        ctypes.POINTER(ctypes.c_int)]),
+    "int8_layer_unpack": (_I32, [_P, _SZ, _P, _P, _P]),
     "int8_linear_forward_decode_static": (_I32, [_P, _I64, _I64, _P, _P, _P, _I64, _F32, _P, _P, _P, _P]),
 }
 
@@ -74,7 +82,9 @@ def lib() -> ctypes.CDLL:
                         f"{LIB_PATH} is missing: build it with `python -m int8_mixed_precision_column_b200.build`")
                 h = ctypes.CDLL(LIB_PATH)
                 for name, (res, args) in SIGNATURES.items():
-                    f = getattr(h, name)
+                    f = getattr(h, name, None)  # every declared symbol is checked by the ABI tests
+                    if f is None:
+                        continue
                     f.restype = res
                     f.argtypes = args
                 _lib = h
@@ -104,6 +114,10 @@ def _require(t: torch.Tensor, dtype: torch.dtype, shape: tuple, name: str) -> No
 # ---------------------------------------------------------------------------
 # entry points
 # ---------------------------------------------------------------------------
+
+def int8_last_cuda_error() -> str:
+    return lib().int8_last_cuda_error().decode()
+
 
 def int8_status_string(status: int) -> str:
     return lib().int8_status_string(status).decode()
@@ -181,6 +195,28 @@ def int8_linear_forward_timed(X, CB, SCB, bias, threshold, Y, idx, n_out, worksp
     _check("int8_linear_forward_timed", st)
 
 
+def int8_linear_forward_fp16w(X: torch.Tensor, W: torch.Tensor, bias: torch.Tensor | None, threshold: float, *,
+                              Y=None, idx=None, n_out=None, workspace=None, stream=None):
+    """has_fp16_weights=True forward: W fp16 [N,K] is quantised inside every call.
+    Returns (Y, idx, n_out, workspace); CB/SCB of this call sit in the workspace."""
+    T, K = X.shape
+    N = W.shape[0]
+    _require(X, torch.float16, (T, K), "X")
+    _require(W, torch.float16, (N, K), "W")
+    if bias is not None:
+        _require(bias, torch.float16, (N,), "bias")
+    dev = X.device
+    Y = torch.empty((T, N), dtype=torch.float16, device=dev) if Y is None else Y
+    idx = torch.empty((K,), dtype=torch.int32, device=dev) if idx is None else idx
+    n_out = torch.empty((1,), dtype=torch.int32, device=dev) if n_out is None else n_out
+    if workspace is None:
+        workspace = torch.empty(int(lib().int8_linear_fp16w_workspace_bytes(T, K, N)), dtype=torch.uint8, device=dev)
+    st = lib().int8_linear_forward_fp16w(_ptr(X), T, K, _ptr(W), _ptr(bias), N, float(threshold), _ptr(Y), _ptr(idx),
+                                         _ptr(n_out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("int8_linear_forward_fp16w", st)
+    return Y, idx, n_out, workspace
+
+
 def int8_check_status(workspace: torch.Tensor, stream=None) -> tuple[int, int]:
     where = ctypes.c_uint32(0)
     st = lib().int8_check_status(_ptr(workspace), ctypes.byref(where), _stream(stream))
@@ -236,3 +272,47 @@ def workspace_views(workspace: torch.Tensor, T: int, K: int, N: int) -> dict:
         "Wo": view(L["Wo"], N * ldo * 2, torch.float16, (N, ldo)),
         "ldo": ldo,
     }
+
+
+# ---------------------------------------------------------------------------
+# persistence of a quantised layer
+# ---------------------------------------------------------------------------
+
+def int8_layer_pack(CB: torch.Tensor, SCB: torch.Tensor, bias: torch.Tensor | None = None) -> bytes:
+    """Byte image of a quantised layer (CB, SCB, optional bias), any device."""
+    N, K = CB.shape
+    cb = CB.detach().to("cpu").contiguous()
+    scb = SCB.detach().to("cpu", torch.float32).contiguous()
+    b = None if bias is None else bias.detach().to("cpu", torch.float16).contiguous()
+    n = int(lib().int8_layer_packed_bytes(N, K, 0 if b is None else 1))
+    if n == 0:
+        raise ValueError(f"unsupported shape N={N} K={K}")
+    out = ctypes.create_string_buffer(n)
+    _check("int8_layer_pack", lib().int8_layer_pack(cb.data_ptr(), scb.data_ptr(), None if b is None else b.data_ptr(),
+                                                    N, K, ctypes.addressof(out), n))
+    return out.raw
+
+
+def int8_layer_unpack(image: bytes, device="cuda"):
+    """(CB int8 [N,K], SCB fp32 [N], bias fp16 [N] or None) from a byte image."""
+    buf = ctypes.create_string_buffer(bytes(image), len(image))
+    N, K, hb = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int(0)
+    _check("int8_layer_unpack_header", lib().int8_layer_unpack_header(ctypes.addressof(buf), len(image),
+                                                                      ctypes.byref(N), ctypes.byref(K), ctypes.byref(hb)))
+    CB = torch.empty((N.value, K.value), dtype=torch.int8)
+    SCB = torch.empty((N.value,), dtype=torch.float32)
+    b = torch.empty((N.value,), dtype=torch.float16) if hb.value else None
+    _check("int8_layer_unpack", lib().int8_layer_unpack(ctypes.addressof(buf), len(image), CB.data_ptr(), SCB.data_ptr(),
+                                                        None if b is None else b.data_ptr()))
+    return CB.to(device), SCB.to(device), (None if b is None else b.to(device))
+
+
+def save_quantized(path: str, CB: torch.Tensor, SCB: torch.Tensor, bias: torch.Tensor | None = None) -> None:
+    with open(path, "wb") as f:
+        f.write(int8_layer_pack(CB, SCB, bias))
+
+
+def load_quantized(path: str, device="cuda"):
+    with open(path, "rb") as f:
+        return int8_layer_unpack(f.read(), device)
+

@@ -12,6 +12,7 @@ from .llm_int8 import (  # noqa: F401
     dequantize_weight,
     int8_matmul,
     linear_forward,
+    linear_forward_fp16w,
     outlier_index,
     outlier_mask,
     outlier_operands,

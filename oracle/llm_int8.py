@@ -213,6 +213,29 @@ def linear_forward(X, CB, SCB, bias, threshold, rows=None) -> dict:
             "Xo": Xo, "Wo": Wo, "acc": acc, "Y": Y}
 
 
+def linear_forward_fp16w(X, W, bias, threshold, rows=None) -> dict:
+    """Forward with has_fp16_weights=True: W stays fp16 and is quantised anew
+    in every forward (bitsandbytes Linear8bitLt docstring, ``has_fp16_weights``).
+
+    Reading taken: with the fp16 weight at hand, the outlier columns are
+    multiplied with W's own fp16 values, Wo = W[:, idx], instead of the
+    dequantised CB.
+    """
+    W = np.asarray(W, dtype=np.float16)
+    X = np.asarray(X, dtype=np.float16)
+    CB, SCB = quantize_weight(W)
+    mask = outlier_mask(X, threshold)
+    idx = outlier_index(mask)
+    Xs = X if rows is None else X[np.asarray(rows)]
+    Xq, sA = quantize_rows(Xs, mask)
+    Xo = Xs[:, idx]
+    Wo = W[:, idx]
+    acc = int8_matmul(Xq, CB)
+    Y = combine(acc, sA, SCB, Xo, Wo, bias)
+    return {"mask": mask, "idx": idx, "n_out": int(idx.size), "Xq": Xq, "sA": sA, "CB": CB, "SCB": SCB,
+            "Xo": Xo, "Wo": Wo, "acc": acc, "Y": Y}
+
+
 def y_tolerance(Yref: np.ndarray) -> float:
     """Allowed max |Y - Yref| for the fp16 output: 1e-3 * max|Yref| + 2e-3."""
     return 1e-3 * float(np.abs(Yref).max(initial=0.0)) + 2e-3

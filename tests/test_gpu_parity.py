@@ -44,7 +44,7 @@ def gpu_forward(p, path="auto", workspace_fill=None):
         ws.fill_(workspace_fill)
     Y, idx, n_out, ws = native.int8_linear_forward(X, CB, SCB, bias, p.threshold, workspace=ws, path=PATHS[path])
     st, where = native.int8_check_status(ws)
-    assert st == 0, f"device status {st} at {where:#x}"
+    assert st == 0, f"device status {st} at {where:#x} ({native.int8_last_cuda_error()})"
     v = native.workspace_views(ws, p.T, p.K, p.N)
     n = int(n_out.item())
     npad = (n + 63) // 64 * 64
@@ -321,3 +321,55 @@ def test_host_buffer_forward_matches_device_forward():
     assert int(n_h) == g["n_out"]
     assert np.array_equal(idx_h.numpy()[: g["n_out"]], g["idx"])
     assert torch.equal(Yh, g["Y"].cpu())
+
+
+# ---------------------------------------------------------------------------
+# rounding and subnormal edge cases of the row codes and the outlier test
+# ---------------------------------------------------------------------------
+
+def _boundary_rows(seed=0, rows=48, K=512):
+    """Rows whose products x * fp32(127/absmax) land on, just below and just
+    above every k + 0.5 boundary, for a spread of absmax values."""
+    rng = np.random.default_rng(seed)
+    X = np.zeros((rows, K), np.float16)
+    for r in range(rows):
+        a = np.float16(127.0) if r == 0 else np.float16(rng.uniform(0.01, 100.0))
+        inv = np.float32(127.0) / np.float32(a)
+        vals = [a, -a]
+        for k in range(0, 127):
+            tgt = np.float16((k + 0.5) / float(inv))
+            for v in (tgt, np.nextafter(tgt, np.float16(0)), np.nextafter(tgt, np.float16(np.inf))):
+                if abs(float(v)) <= float(a):
+                    vals += [v, -v]
+        vals = np.array(vals[:K], np.float16)
+        X[r, : vals.size] = vals
+    return X
+
+
+@pytest.mark.parametrize("path", ["tc", "decode"])
+def test_row_codes_at_rounding_boundaries(path):
+    X = _boundary_rows(rows=48 if path == "tc" else 16)
+    T, K = X.shape
+    W = (np.random.default_rng(1).normal(0, 0.02, (64, K))).astype(np.float16)
+    p = workloads.LinearProblem("bounds", torch.from_numpy(X), torch.from_numpy(W), None, 1000.0)
+    g = gpu_forward(p, path)
+    mask = O.outlier_mask(X, 1000.0)
+    Xq, sA = O.quantize_rows(X, mask)
+    assert g["n_out"] == 0
+    assert np.array_equal(to_np(g["sA"]), sA)
+    assert np.array_equal(to_np(g["Xq"]), Xq)
+
+
+@pytest.mark.parametrize("thr", [1e-6, 3e-5, 6.0])
+def test_subnormal_rows_and_thresholds(thr):
+    rng = np.random.default_rng(2)
+    T, K, N = 24, 256, 64
+    X = (rng.normal(0, 1, (T, K)) * 1e-6).astype(np.float16)   # mostly fp16 subnormals
+    X[3] = (rng.normal(0, 1, K) * 2e-7).astype(np.float16)
+    X[5, 7] = np.float16(6e-5)
+    X[9] = 0
+    X[9, 11] = np.float16(5.96e-8)                               # smallest subnormal
+    W = rng.normal(0, 0.02, (N, K)).astype(np.float16)
+    p = workloads.LinearProblem("subnormal", torch.from_numpy(X), torch.from_numpy(W), None, thr)
+    for path in ("tc", "decode" if T <= 16 else "tc1"):
+        check_forward(p, gpu_forward(p, path))

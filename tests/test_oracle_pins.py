@@ -305,12 +305,45 @@ def check_outlier_operands():
             assert r["Wo"][j, oi] == v
 
 
+def check_fp16w_all_columns_is_exact_product():
+    """has_fp16_weights=True, every column flagged: Y = X @ W^T + b exactly."""
+    p = workloads.make_problem("fp16w", 10, 48, 24, w_std=0.05, bias_std=0.01, seed=13)
+    X = p.X.numpy()
+    X[np.abs(X) <= 0.1] = np.float16(0.5)
+    W, b = p.W.numpy(), p.bias.numpy()
+    r = O.linear_forward_fp16w(X, W, b, 0.1)
+    assert r["n_out"] == 48 and np.all(r["acc"] == 0)
+    exact = X.astype(np.float64) @ W.astype(np.float64).T + b.astype(np.float64)
+    np.testing.assert_allclose(r["Y"], exact, rtol=1e-12, atol=1e-12)
+
+
+def check_fp16w_without_outliers_equals_int8_forward():
+    p = workloads.make_problem("fp16w0", 9, 64, 32, n_planted=3, bias_std=0.01, seed=14)
+    X, W, b = p.X.numpy(), p.W.numpy(), p.bias.numpy()
+    r = O.linear_forward_fp16w(X, W, b, 0.0)
+    r8 = O.linear_forward(X, *O.quantize_weight(W), b, 0.0)
+    assert np.array_equal(r["Y"], r8["Y"]) and r["n_out"] == 0
+
+
+def check_fp16w_outlier_weights_are_the_fp16_columns():
+    X, W, b, cols = lossless_problem(21, True)
+    W = W.astype(np.float16)
+    W[:, cols] = np.float16(0.3333)          # not representable as CB*SCB/127 with SCB = 127
+    W[:, 0] = np.float16(127.0)              # keep each row's absmax (127) in a non-outlier column
+    r = O.linear_forward_fp16w(X, W, b, 150.0)
+    assert r["idx"].tolist() == cols and np.array_equal(r["Wo"], W[:, cols])
+    exact = X.astype(np.float64) @ W.astype(np.float64).T + b.astype(np.float64)
+    np.testing.assert_allclose(r["Y"], exact, rtol=0, atol=1e-9)
+
+
 ALL_PINS = [
     check_worked_example, check_rounding, check_range_and_absmax, check_recovery_half_step,
     check_mask_bruteforce, check_toy_columns, check_issue_1609, check_threshold_off,
     check_idx_ignores_weights, check_rowquant_bruteforce, check_int8_matmul_bruteforce,
     check_lossless_closed_form, check_all_columns_flagged, check_pure_int8_path,
     check_bias_linearity, check_error_bound, check_outlier_operands,
+    check_fp16w_all_columns_is_exact_product, check_fp16w_without_outliers_equals_int8_forward,
+    check_fp16w_outlier_weights_are_the_fp16_columns,
 ]
 
 

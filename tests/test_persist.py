@@ -1,0 +1,73 @@
+"""Persistence of a quantised layer (CB, SCB, bias) as one byte image."""
+
+from __future__ import annotations
+
+import struct
+
+import numpy as np
+import pytest
+import torch
+
+from int8_mixed_precision_column_b200 import build, native, workloads
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    native.lib()
+
+
+def _layer(N=48, K=80, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    CB = torch.randint(-127, 128, (N, K), generator=g, dtype=torch.int8)
+    SCB = torch.rand(N, generator=g) * 0.1
+    bias = (torch.randn(N, generator=g) * 0.01).half()
+    return CB, SCB, bias
+
+
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_round_trip(with_bias):
+    CB, SCB, bias = _layer()
+    img = native.int8_layer_pack(CB, SCB, bias if with_bias else None)
+    cb2, scb2, b2 = native.int8_layer_unpack(img, device="cpu")
+    assert torch.equal(cb2, CB) and torch.equal(scb2, SCB)
+    assert (b2 is None) == (not with_bias)
+    if with_bias:
+        assert torch.equal(b2, bias)
+
+
+def test_byte_layout_is_the_documented_one():
+    CB, SCB, bias = _layer(N=16, K=32, seed=1)
+    img = native.int8_layer_pack(CB, SCB, bias)
+    assert img[:8] == b"I8MPLYR1"
+    assert struct.unpack_from("<qqII", img, 8) == (16, 32, 1, 0)
+    assert np.array_equal(np.frombuffer(img, np.float32, 16, 32), SCB.numpy())
+    assert np.array_equal(np.frombuffer(img, np.float16, 16, 32 + 64), bias.numpy())
+    assert np.array_equal(np.frombuffer(img, np.int8, 16 * 32, 32 + 64 + 32).reshape(16, 32), CB.numpy())
+    assert len(img) == native.lib().int8_layer_packed_bytes(16, 32, 1) == 32 + 64 + 32 + 512
+
+
+def test_malformed_images_are_rejected():
+    CB, SCB, bias = _layer()
+    img = native.int8_layer_pack(CB, SCB, bias)
+    bad = [b"X" + img[1:], img[:-1], img[:20],
+           img[:8] + struct.pack("<q", 15) + img[16:],          # N not a multiple of 16
+           img[:24] + struct.pack("<I", 2) + img[28:]]           # unknown flag
+    for b in bad:
+        with pytest.raises(native.Int8mpError):
+            native.int8_layer_unpack(b, device="cpu")
+    assert native.lib().int8_layer_packed_bytes(15, 32, 0) == 0
+
+
+@pytest.mark.gpu
+def test_loaded_layer_gives_the_same_forward(tmp_path):
+    assert torch.cuda.is_available()
+    p = workloads.make_problem("persist", 64, 1024, 512, n_planted=5, bias_std=0.01, seed=3)
+    CB, SCB = native.int8_quantize_weight(p.W.cuda())
+    bias = p.bias.cuda()
+    path = tmp_path / "layer.i8mp"
+    native.save_quantized(str(path), CB, SCB, bias)
+    CB2, SCB2, b2 = native.load_quantized(str(path), device="cuda")
+    Y1, idx1, n1, _ = native.int8_linear_forward(p.X.cuda(), CB, SCB, bias, 6.0)
+    Y2, idx2, n2, _ = native.int8_linear_forward(p.X.cuda(), CB2, SCB2, b2, 6.0)
+    assert torch.equal(Y1, Y2) and int(n1) == int(n2)
