@@ -64,6 +64,38 @@ def load_peaks() -> tuple[dict, str]:
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# Kernel source files each measured kernel is built from: a DRAM-traffic figure
+# recorded in profiles/traffic.json is reported only while these are unchanged.
+KERNEL_SOURCES = {
+    "gemm_i8_tc2_kernel": ["gemm_tc2.cu", "common.cuh", "kernels.h"],
+    "gemm_i8_tc_kernel": ["gemm_tc.cu", "common.cuh", "kernels.h"],
+    "gemv_i8_decode_kernel": ["gemv_decode.cu", "common.cuh", "kernels.h"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "int8_mixed_precision_column_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, workload: str) -> tuple[float | None, str]:
+    """DRAM bytes per launch from an ncu capture committed under profiles/, or None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None, "no capture recorded"
+    with open(path) as f:
+        rec = json.load(f).get(kernel, {}).get(workload)
+    if rec is None:
+        return None, "no capture for this kernel and workload"
+    if rec.get("source_sha256") != kernel_source_hash(kernel):
+        return None, "kernel changed since the capture"
+    return float(rec["dram_bytes_per_launch"]), rec.get("command", "")
+
+
 def dist_env() -> tuple[int, int, int]:
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
@@ -193,13 +225,19 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     if args.threshold is not None:
         p.threshold = args.threshold
     T, K, N = p.T, p.K, p.N
+    cpu_sample = sample_problem(p, 256, 4096) if (world == 1 and not args.no_cpu_baseline) else None
+    elem = torch.bfloat16 if args.dtype == "bf16" else torch.float16
+    if elem != torch.float16:
+        # the same seeded problem, rounded to bf16 (X, W, bias)
+        p.X, p.W = p.X.to(elem), p.W.to(elem)
+        p.bias = None if p.bias is None else p.bias.to(elem)
+        cpu_sample = None
     bias = p.bias
     CB, SCB = native.int8_quantize_weight(p.W)
-    cpu_sample = sample_problem(p, 256, 4096) if (world == 1 and not args.no_cpu_baseline) else None
     del p.W
     torch.cuda.empty_cache()
     X = p.X
-    Y = torch.empty((T, N), dtype=torch.float16, device=dev)
+    Y = torch.empty((T, N), dtype=elem, device=dev)
     idx = torch.empty((K,), dtype=torch.int32, device=dev)
     n_out = torch.empty((1,), dtype=torch.int32, device=dev)
     ws = native.new_workspace(T, K, N, dev)
@@ -257,7 +295,7 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
 
     # end to end through the host-buffer entry point: pinned X in, Y/idx/n_out out, per step
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and elem == torch.float16:  # the host-buffer entry point takes fp16
         Xh = X.cpu().pin_memory()
         Yh = torch.empty((T, N), dtype=torch.float16).pin_memory()
         idx_h = torch.empty((K,), dtype=torch.int32).pin_memory()
@@ -290,18 +328,24 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     peaks, peak_src = load_peaks()
     prod_avg = statistics.mean(prod_ms)
     decode = T <= 16 if args.path == 0 else args.path == 2
+    traffic_key = args.workload if elem == torch.float16 else f"{args.workload}_bf16"
     if decode:
         achieved = work["product_bytes"] / (prod_avg * 1e-3) / 1e9
+        traffic, traffic_src = recorded_traffic("gemv_i8_decode_kernel", traffic_key)
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "gemv_i8_decode_kernel",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "traffic_source": traffic_src,
+                "kernel": "gemv_i8_decode_kernel",
                 "peak_source": f"{peak_src} hbm_gbs (copy)",
                 "algorithmic_bytes_per_launch": work["product_bytes"], "ms_per_launch": prod_avg}
     else:
         peak = peaks["bf16_tflops"] * INT8_PER_BF16
         achieved = work["int8_ops"] / (prod_avg * 1e-3) / 1e12
+        kname = "gemm_i8_tc_kernel" if args.path == 3 else "gemm_i8_tc2_kernel"
+        traffic, traffic_src = recorded_traffic(kname, traffic_key)
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS",
-                "frac": achieved / peak, "traffic": None,
-                "kernel": "gemm_i8_tc_kernel" if args.path == 3 else "gemm_i8_tc2_kernel",
+                "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
+                "algorithmic_bytes_per_launch": work["product_bytes"],
+                "kernel": kname,
                 "peak_source": f"{peak_src} bf16_tflops (burst) x {INT8_PER_BF16} nominal int8:bf16 ratio",
                 "algorithmic_ops_per_launch": work["int8_ops"], "ms_per_launch": prod_avg}
     launches_per_step = 3 if p.threshold > 0 else 2
@@ -318,9 +362,10 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int8 x int8 -> int32 (+ fp16 outlier product, fp32 accumulate), fp16 in/out",
+        "dtype": f"int8 x int8 -> int32 (+ {args.dtype} outlier product, fp32 accumulate), {args.dtype} in/out",
         "data": "synthetic (seeded; X ~ N(0,1) with planted outlier columns, W ~ N(0, 0.02^2))",
         "config": {"workload": args.workload, "T": T, "K": K, "N": N, "threshold": p.threshold, "path": args.path,
+                   "elem": args.dtype,
                    "n_out": n_outliers, "parallelism": f"independent problem per rank x{world}",
                    "l2": "L2 flushed between steps" if flush else "inputs larger than L2 (no flush)"},
         "stage_ms": {"outliers": statistics.mean(outl_ms), "rowquant": statistics.mean(rowq_ms),
@@ -431,6 +476,8 @@ def main() -> None:
                     help="override the workload's outlier threshold (<= 0 switches the decomposition off)")
     ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2, 3],
                     help="product kernel: 0 auto, 1 tensor core (SM pairs), 2 decode GEMV, 3 tensor core (single SM)")
+    ap.add_argument("--dtype", default="fp16", choices=["fp16", "bf16"],
+                    help="16-bit element type of X, bias, Y and the outlier product")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

@@ -246,6 +246,46 @@ i8_status int8_selftest_wait_timeout(void* workspace, size_t workspace_bytes, ui
 uint32_t int8_outlier_threshold_bits(float threshold);
 
 /* ---------------------------------------------------------------------------
+ * 16-bit element type.
+ *
+ * The bitsandbytes Linear8bitLt docstring describes the module for fp16 or
+ * bf16 weights; the calls above take fp16.  The calls below take the element
+ * type of every 16-bit operand -- X, W, bias, Y and the internal outlier
+ * operands -- as `dtype`: I8_DTYPE_F16 (the calls above) or I8_DTYPE_BF16.
+ * With bf16 the outlier test compares bf16 magnitudes, the outlier product
+ * multiplies bf16 operands (the dequantised outlier weights are rounded to
+ * bf16) with fp32 accumulation, and Y is rounded to bf16 (round to nearest
+ * even).  The int8 stages and the fp32 arithmetic are those of the fp16 path.
+ * Any other dtype value is I8_ERR_INVALID_ARG.
+ * ------------------------------------------------------------------------- */
+enum { I8_DTYPE_F16 = 0, I8_DTYPE_BF16 = 1 };
+
+/* int8_quantize_weight with W of element type `dtype`. */
+i8_status int8_quantize_weight_ex(const void* W, int dtype, int64_t N, int64_t K, int8_t* CB, float* SCB,
+                                  cudaStream_t stream);
+
+/* The forward with X, bias and Y of element type `dtype`, the product kernel
+ * chosen by `path` (as int8_linear_forward_path) and, when `events` is not
+ * NULL, the four stage events of int8_linear_forward_timed.  Workspace size,
+ * arguments, results and errors as int8_linear_forward. */
+i8_status int8_linear_forward_ex(const void* X, int dtype, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                                 const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
+                                 int32_t* n_out, void* workspace, size_t workspace_bytes, int path,
+                                 void* const* events, cudaStream_t stream);
+
+/* int8_linear_forward_fp16w (has_fp16_weights=True) with X, W, bias and Y of
+ * element type `dtype`. */
+i8_status int8_linear_forward_fp16w_ex(const void* X, int dtype, int64_t T, int64_t K, const void* W,
+                                       const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
+                                       int32_t* n_out, void* workspace, size_t workspace_bytes,
+                                       cudaStream_t stream);
+
+/* int8_outlier_threshold_bits for element type `dtype`: the largest magnitude
+ * pattern of that type (bf16: 0..0x7f80) whose value is <= threshold.
+ * 0xffffffff when threshold <= 0 or NaN, 0xfffffffe for an unknown dtype. */
+uint32_t int8_outlier_threshold_bits_ex(float threshold, int dtype);
+
+/* ---------------------------------------------------------------------------
  * Forward without any caller-provided or allocated scratch memory.
  *
  * The pages have no counterpart to this call: it exists for callers that

@@ -85,19 +85,30 @@ float half_bits_value(uint32_t h) {
   return std::ldexp(static_cast<float>(m | 0x400u), static_cast<int>(e) - 25);
 }
 
-uint32_t threshold_bits(float thr) {
+// bf16 is the upper half of an fp32 pattern.
+float bf16_bits_value(uint32_t h) {
+  const uint32_t u = h << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+uint32_t threshold_bits(float thr, int dtype = kF16) {
   if (!(thr > 0.0f)) return 0xffffffffu;
-  // largest pattern p in [0, 0x7c00] with value(p) <= thr; value is monotone in p.
-  uint32_t lo = 0, hi = 0x7c00;
+  // largest pattern p in [0, inf pattern] with value(p) <= thr; value is monotone in p.
+  const bool bf = dtype == kBF16;
+  uint32_t lo = 0, hi = bf ? 0x7f80u : 0x7c00u;
   while (lo < hi) {
     const uint32_t mid = (lo + hi + 1) / 2;
-    if (half_bits_value(mid) <= thr)
+    if ((bf ? bf16_bits_value(mid) : half_bits_value(mid)) <= thr)
       lo = mid;
     else
       hi = mid - 1;
   }
   return lo;
 }
+
+inline bool dtype_ok(int dtype) { return dtype == kF16 || dtype == kBF16; }
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
@@ -118,8 +129,9 @@ cudaError_t launch_product(const GemmArgs& a, int path, bool gemv, int num_sms, 
 
 i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB, const void* bias,
                        int64_t N, float threshold, void* Y, int32_t* idx, int32_t* n_out, void* ws, size_t ws_bytes,
-                       int path, void* const* events, cudaStream_t stream, const __half* Wf = nullptr) {
-  if (!shape_ok(T, K, N)) return I8_ERR_INVALID_ARG;
+                       int path, void* const* events, cudaStream_t stream, int dtype = kF16,
+                       const void* Wf = nullptr) {
+  if (!shape_ok(T, K, N) || !dtype_ok(dtype)) return I8_ERR_INVALID_ARG;
   if (path < kPathAuto || path > kPathTensorCoreSingleSM) return I8_ERR_INVALID_ARG;
   if (path == kPathDecode && T > kDecodeMaxT) return I8_ERR_INVALID_ARG;
   if (idx == nullptr || n_out == nullptr || !aligned(idx, 4) || !aligned(n_out, 4)) return I8_ERR_INVALID_ARG;
@@ -154,21 +166,20 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   uint32_t* prefix = mask + (K + 31) / 32;
   float* sA = reinterpret_cast<float*>(w + L.sA);
   int8_t* Xq = reinterpret_cast<int8_t*>(w + L.Xq);
-  __half* Xo = reinterpret_cast<__half*>(w + L.Xo);
-  __half* Wo = reinterpret_cast<__half*>(w + L.Wo);
-  const __half* Xh = static_cast<const __half*>(X);
+  void* Xo = w + L.Xo;
+  void* Wo = w + L.Wo;
 
-  const uint32_t hb = threshold_bits(threshold);
+  const uint32_t hb = threshold_bits(threshold, dtype);
   if (hb == 0xffffffffu)
     e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
   else
-    e = launch_outliers(Xh, T, K, hb, mask, prefix, idx, n_out, dst, stream);
+    e = launch_outliers(X, dtype, T, K, hb, mask, prefix, idx, n_out, dst, stream);
   if (e != cudaSuccess || !mark(1)) return I8_ERR_CUDA;
 
   const bool gemv = (path == kPathDecode) || (path == kPathAuto && T <= kDecodeMaxT);
   // programmatic launches only directly after one of our kernels
   const bool after_outliers = (hb != 0xffffffffu);
-  e = launch_rowquant(Xh, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, Wf, num_sms,
+  e = launch_rowquant(X, dtype, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, Wf, num_sms,
                       dst, after_outliers, stream);
   if (e != cudaSuccess || !mark(2)) return I8_ERR_CUDA;
 
@@ -180,8 +191,8 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   a.ldo = L.ldo;
   a.sA = sA;
   a.SCB = SCB;
-  a.bias = static_cast<const __half*>(bias);
-  a.Y = static_cast<__half*>(Y);
+  a.bias = bias;
+  a.Y = Y;
   a.acc_out = nullptr;
   a.n_out = n_out;
   a.idx = idx;
@@ -192,6 +203,7 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   a.mode = 0;
   a.pdl = true;  // follows the row quantisation kernel
   a.Wf = Wf;
+  a.dtype = dtype;
   e = launch_product(a, path, gemv, num_sms, stream);
   if (e != cudaSuccess || !mark(3)) return I8_ERR_CUDA;
   return I8_OK;
@@ -215,9 +227,16 @@ const char* int8_status_string(int status) {
 
 int int8_version(void) { return 100; }
 
-uint32_t int8_outlier_threshold_bits(float threshold) { return threshold_bits(threshold); }
+uint32_t int8_outlier_threshold_bits(float threshold) { return threshold_bits(threshold, kF16); }
 
-i8_status int8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* CB, float* SCB, cudaStream_t stream) {
+uint32_t int8_outlier_threshold_bits_ex(float threshold, int dtype) {
+  if (!dtype_ok(dtype)) return 0xfffffffeu;
+  return threshold_bits(threshold, dtype);
+}
+
+i8_status int8_quantize_weight_ex(const void* W, int dtype, int64_t N, int64_t K, int8_t* CB, float* SCB,
+                                  cudaStream_t stream) {
+  if (!dtype_ok(dtype)) return I8_ERR_INVALID_ARG;
   if (N < 0 || N > kMaxRows || K < 16 || K % 16 != 0 || K > kMaxK) return I8_ERR_INVALID_ARG;
   if (N == 0) return I8_OK;
   if (W == nullptr || CB == nullptr || SCB == nullptr) return I8_ERR_INVALID_ARG;
@@ -225,7 +244,11 @@ i8_status int8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* CB, 
   int num_sms = 0;
   i8_status st = device_info(&num_sms);
   if (st != I8_OK) return st;
-  return cuda_status(launch_quantize_weight(static_cast<const __half*>(W), N, K, CB, SCB, stream));
+  return cuda_status(launch_quantize_weight(W, dtype, N, K, CB, SCB, stream));
+}
+
+i8_status int8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* CB, float* SCB, cudaStream_t stream) {
+  return int8_quantize_weight_ex(W, kF16, N, K, CB, SCB, stream);
 }
 
 size_t int8_linear_workspace_bytes(int64_t T, int64_t K, int64_t N) {
@@ -265,6 +288,17 @@ i8_status int8_linear_forward_timed(const void* X, int64_t T, int64_t K, const i
                       stream);
 }
 
+i8_status int8_linear_forward_ex(const void* X, int dtype, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                                 const void* bias, int64_t N, float threshold, void* Y, int32_t* idx, int32_t* n_out,
+                                 void* workspace, size_t workspace_bytes, int path, void* const* events,
+                                 cudaStream_t stream) {
+  if (events != nullptr)
+    for (int i = 0; i < 4; ++i)
+      if (events[i] == nullptr) return I8_ERR_INVALID_ARG;
+  return forward_impl(X, T, K, CB, SCB, bias, N, threshold, Y, idx, n_out, workspace, workspace_bytes, path, events,
+                      stream, dtype);
+}
+
 i8_status int8_check_status(void* workspace, uint32_t* where, cudaStream_t stream) {
   if (workspace == nullptr || !aligned(workspace, 256)) return I8_ERR_WORKSPACE;
   if (where != nullptr) *where = 0xffffffffu;  // "the synchronisation itself failed"
@@ -291,10 +325,10 @@ size_t int8_linear_fp16w_workspace_bytes(int64_t T, int64_t K, int64_t N) {
   return static_cast<size_t>(align_up(align_up(L.total + static_cast<uint64_t>(N) * K, 256) + N * 4, 256));
 }
 
-i8_status int8_linear_forward_fp16w(const void* X, int64_t T, int64_t K, const void* W, const void* bias, int64_t N,
-                                    float threshold, void* Y, int32_t* idx, int32_t* n_out, void* workspace,
-                                    size_t workspace_bytes, cudaStream_t stream) {
-  if (!shape_ok(T, K, N)) return I8_ERR_INVALID_ARG;
+i8_status int8_linear_forward_fp16w_ex(const void* X, int dtype, int64_t T, int64_t K, const void* W,
+                                       const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
+                                       int32_t* n_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!shape_ok(T, K, N) || !dtype_ok(dtype)) return I8_ERR_INVALID_ARG;
   if (W == nullptr || !aligned(W, 16)) return I8_ERR_INVALID_ARG;
   const int8_ws_layout L = make_layout(T, K, N);
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < int8_linear_fp16w_workspace_bytes(T, K, N))
@@ -306,9 +340,16 @@ i8_status int8_linear_forward_fp16w(const void* X, int64_t T, int64_t K, const v
   i8_status st = device_info(&num_sms);
   if (st != I8_OK) return st;
   // the weight is quantised anew in every forward (Linear8bitLt, has_fp16_weights=True)
-  if (launch_quantize_weight(static_cast<const __half*>(W), N, K, CB, SCB, stream) != cudaSuccess) return I8_ERR_CUDA;
+  if (launch_quantize_weight(W, dtype, N, K, CB, SCB, stream) != cudaSuccess) return I8_ERR_CUDA;
   return forward_impl(X, T, K, CB, SCB, bias, N, threshold, Y, idx, n_out, workspace, L.total, 0, nullptr, stream,
-                      static_cast<const __half*>(W));
+                      dtype, W);
+}
+
+i8_status int8_linear_forward_fp16w(const void* X, int64_t T, int64_t K, const void* W, const void* bias, int64_t N,
+                                    float threshold, void* Y, int32_t* idx, int32_t* n_out, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
+  return int8_linear_forward_fp16w_ex(X, kF16, T, K, W, bias, N, threshold, Y, idx, n_out, workspace,
+                                      workspace_bytes, stream);
 }
 
 size_t int8_linear_forward_host_workspace_bytes(int64_t T, int64_t K, int64_t N) {

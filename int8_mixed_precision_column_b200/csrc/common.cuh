@@ -4,10 +4,67 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace i8mp {
+
+// ---------------------------------------------------------------------------
+// 16-bit element types of activations, bias, outlier operands and output:
+// fp16 (the default) or bf16 (the module is documented for fp16 / bf16).
+// ---------------------------------------------------------------------------
+enum DType : int { kF16 = 0, kBF16 = 1 };
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<__half> {
+  using T2 = __half2;
+  static constexpr uint32_t kInfBits = 0x7c00u;  // magnitude pattern of +inf
+  static constexpr uint32_t kMmaFormat = 0;      // tcgen05 kind::f16 operand format: F16
+  __device__ static __forceinline__ float to_float(__half h) { return __half2float(h); }
+  __device__ static __forceinline__ __half from_float(float f) { return __float2half_rn(f); }
+  __device__ static __forceinline__ float2 to_float2(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
+  }
+  __device__ static __forceinline__ uint32_t pack2(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  // elementwise max of two pairs of non-negative values (a NaN operand is ignored)
+  __device__ static __forceinline__ uint32_t max2(uint32_t a, uint32_t b) {
+    __half2 m = __hmax2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&m);
+  }
+  // value of a magnitude pattern
+  __device__ static __forceinline__ float mag_to_float(uint32_t bits) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
+  }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+  using T2 = __nv_bfloat162;
+  static constexpr uint32_t kInfBits = 0x7f80u;
+  static constexpr uint32_t kMmaFormat = 1;      // BF16
+  __device__ static __forceinline__ float to_float(__nv_bfloat16 h) { return __bfloat162float(h); }
+  __device__ static __forceinline__ __nv_bfloat16 from_float(float f) { return __float2bfloat16_rn(f); }
+  __device__ static __forceinline__ float2 to_float2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  }
+  __device__ static __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __device__ static __forceinline__ uint32_t max2(uint32_t a, uint32_t b) {
+    __nv_bfloat162 m =
+        __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a), *reinterpret_cast<const __nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&m);
+  }
+  __device__ static __forceinline__ float mag_to_float(uint32_t bits) { return __uint_as_float(bits << 16); }
+};
 
 // ---------------------------------------------------------------------------
 // Device status word (first 64 bytes of the workspace).
@@ -234,8 +291,9 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
 __host__ __device__ constexpr uint32_t idesc_i8_s32(uint32_t M, uint32_t N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
-__host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t M, uint32_t N) {
-  return (1u << 4) | (0u << 7) | (0u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t M, uint32_t N, uint32_t fmt = 0) {
+  // fmt: 0 = both operands fp16, 1 = both bf16 (A and B always share a type)
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 

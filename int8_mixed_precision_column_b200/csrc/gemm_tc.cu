@@ -3,7 +3,7 @@
 // Computes, per output tile of 128 tokens x 256 output features,
 //   acc[t,j] = sum_k Xq[t,k] * CB[j,k]                 (tcgen05 kind::i8, int32 in TMEM)
 //   Yo[t,j]  = sum_o Xo[t,o] * Wo[j,o]                 (tcgen05 kind::f16, fp32 in TMEM)
-//   Y[t,j]   = fp16(acc * sA[t] * SCB[j] / 127^2 + Yo + bias[j])
+//   Y[t,j]   = TE(acc * sA[t] * SCB[j] / 127^2 + Yo + bias[j])   (TE: fp16 or bf16)
 // i.e. steps 2 and 3 of "Core idea of LLM.int8()" on the Hugging Face
 // integration page (int8 vector-wise product for the bulk, 16-bit product for
 // the outlier columns, dequantise and sum), with the vector-wise constants of
@@ -17,7 +17,7 @@
 //               share the ring and the 128-byte swizzle layout.
 //   warp 1      TMEM allocation (512 columns) and the single MMA-issuing thread.
 //   warps 2..9  epilogue: tcgen05.ld of the accumulators, dequant + outlier
-//               + bias, fp16 stores.
+//               + bias, 16-bit stores.
 // TMEM use: with no outlier columns, two int32 accumulators (columns 0 and 256)
 // let the epilogue of one tile overlap the main loop of the next; with outlier
 // columns, columns 0..255 hold the int32 and 256..511 the fp32 accumulator.
@@ -43,7 +43,6 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
 constexpr int GROUP_M = 16;  // m-tiles per raster group
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_I8 = idesc_i8_s32(BM, BN);
-constexpr uint32_t IDESC_F16 = idesc_f16_f32(BM, BN);
 
 // wait tags reported in DevStatus::where
 constexpr uint32_t W_EMPTY = 0x101, W_FULL = 0x102, W_TEMPTY = 0x103, W_TFULL = 0x104, W_DRAIN = 0x105,
@@ -54,8 +53,8 @@ struct Params {
   int nkb_i8;
   const float* sA;
   const float* SCB;
-  const __half* bias;
-  __half* Y;
+  const void* bias;  // TE[N] or null
+  void* Y;           // TE[T,N]
   int32_t* acc_out;
   const int32_t* n_out;
   DevStatus* st;
@@ -72,15 +71,12 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int&
   n_blk = local / gm;
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
+template <typename TE>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_i8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmAo, const __grid_constant__ CUtensorMap tmBo,
                       const Params p) {
+  constexpr uint32_t kIdescO = idesc_f16_f32(BM, BN, Elem<TE>::kMmaFormat);  // 16-bit outlier MMA
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
@@ -208,7 +204,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int ko = kb - p.nkb_i8;
             #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_f16(d_f32, adesc + 2u * kk, bdesc + 2u * kk, IDESC_F16, (ko | kk) != 0 ? 1u : 0u);
+              mma_f16(d_f32, adesc + 2u * kk, bdesc + 2u * kk, kIdescO, (ko | kk) != 0 ? 1u : 0u);
           }
           mma_commit(&empty_bar[s]);
           if (++s == STAGES) {
@@ -260,7 +256,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         const int64_t my_col = gcol0 + lane;
         const float scb_l = (my_col < p.N) ? __ldg(&p.SCB[my_col]) : 0.0f;
-        const float b_l = (p.bias != nullptr && my_col < p.N) ? __half2float(p.bias[my_col]) : 0.0f;
+        const float b_l = (p.bias != nullptr && my_col < p.N) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[my_col]) : 0.0f;
         uint32_t packed[16];
         #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -274,10 +270,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             y0 += __uint_as_float(fo[i]);
             y1 += __uint_as_float(fo[i + 1]);
           }
-          packed[i >> 1] = pack_half2(y0, y1);
+          packed[i >> 1] = Elem<TE>::pack2(y0, y1);
         }
         if (row_ok) {
-          __half* dst = p.Y + row * p.N + gcol0;
+          TE* dst = static_cast<TE*>(p.Y) + row * p.N + gcol0;
           #pragma unroll
           for (int g = 0; g < 4; ++g)
             if (gcol0 + g * 8 + 8 <= p.N)
@@ -342,7 +338,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t s) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !attr_done[dev]) {
-    e = cudaFuncSetAttribute(gemm_i8_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    e = cudaFuncSetAttribute(gemm_i8_tc_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gemm_i8_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
@@ -351,10 +350,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t s) {
   if (!make_map(&tmA, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.K, a.T, a.K, BKB, BM)) return cudaErrorInvalidValue;
   if (!make_map(&tmB, a.CB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.K, a.N, a.K, BKB, BN)) return cudaErrorInvalidValue;
   const bool outl = a.mode == 0 && a.n_out != nullptr && a.Xo != nullptr && a.Wo != nullptr;
+  const CUtensorMapDataType t16 = a.dtype == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   if (outl) {
-    if (!make_map(&tmAo, a.Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.ldo, a.T, a.ldo * 2, 64, BM))
-      return cudaErrorInvalidValue;
-    if (!make_map(&tmBo, a.Wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.ldo, a.N, a.ldo * 2, 64, BN))
+    if (!make_map(&tmAo, a.Xo, t16, 2, a.ldo, a.T, a.ldo * 2, 64, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&tmBo, a.Wo, t16, 2, a.ldo, a.N, a.ldo * 2, 64, BN))
       return cudaErrorInvalidValue;
   } else {
     tmAo = tmA;  // never read: the kernel runs no outlier K-blocks
@@ -386,7 +385,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel, tmA, tmB, tmAo, tmBo, p);
+  if (a.dtype == kBF16) return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel<__nv_bfloat16>, tmA, tmB, tmAo, tmBo, p);
+  return cudaLaunchKernelEx(&cfg, gemm_i8_tc_kernel<__half>, tmA, tmB, tmAo, tmBo, p);
 }
 
 }  // namespace i8mp

@@ -38,7 +38,6 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
 constexpr int GROUP_M = 8;  // pair tiles (256 rows) per raster group
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_I8 = idesc_i8_s32(2 * BM, BN);
-constexpr uint32_t IDESC_F16 = idesc_f16_f32(2 * BM, BN);
 constexpr uint16_t PAIR_MASK = 0x3;
 
 constexpr uint32_t W_EMPTY = 0x201, W_FULL = 0x202, W_TEMPTY = 0x203, W_TFULL = 0x204, W_DRAIN = 0x205,
@@ -49,14 +48,14 @@ struct Params {
   int nkb_i8;
   const float* sA;
   const float* SCB;
-  const __half* bias;
-  __half* Y;
+  const void* bias;  // TE[N] or null
+  void* Y;           // TE[T,N]
   int32_t* acc_out;
   const int32_t* n_out;
   DevStatus* st;
   int mode;
   int vec_scb;   // SCB is 16-byte aligned: a tile's 16 column scales load as 4 x float4
-  int vec_bias;  // bias is 16-byte aligned: 16 halves load as 2 x uint4
+  int vec_bias;  // bias is 16-byte aligned: 16 elements load as 2 x uint4
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
@@ -69,15 +68,12 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int&
   n_blk = local / gm;
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
+template <typename TE>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_i8_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmAo, const __grid_constant__ CUtensorMap tmBo,
                        const Params p) {
+  constexpr uint32_t kIdescO = idesc_f16_f32(2 * BM, BN, Elem<TE>::kMmaFormat);  // 16-bit outlier MMA
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];   // used in the leader only
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
@@ -216,7 +212,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int ko = kb - p.nkb_i8;
             #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_f16_pair(d_f32, adesc + 2u * kk, bdesc + 2u * kk, IDESC_F16, (ko | kk) != 0 ? 1u : 0u);
+              mma_f16_pair(d_f32, adesc + 2u * kk, bdesc + 2u * kk, kIdescO, (ko | kk) != 0 ? 1u : 0u);
           }
           mma_commit_pair(&empty_bar[s], PAIR_MASK);
           if (++s == STAGES) {
@@ -287,21 +283,22 @@ __global__ void __launch_bounds__(THREADS, 1)
           #pragma unroll
           for (int i = 0; i < 16; ++i) bi[i] = 0.0f;
         } else if (full && p.vec_bias) {
-          const uint4* b8 = reinterpret_cast<const uint4*>(p.bias + gcol0);
+          const uint4* b8 = reinterpret_cast<const uint4*>(static_cast<const TE*>(p.bias) + gcol0);
           #pragma unroll
           for (int q8 = 0; q8 < 2; ++q8) {
             const uint4 v = __ldg(b8 + q8);
-            const __half2* h = reinterpret_cast<const __half2*>(&v);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 f = __half22float2(h[e]);
+              const float2 f = Elem<TE>::to_float2(w[e]);
               bi[8 * q8 + 2 * e] = f.x;
               bi[8 * q8 + 2 * e + 1] = f.y;
             }
           }
         } else {
           #pragma unroll
-          for (int i = 0; i < 16; ++i) bi[i] = (gcol0 + i < p.N) ? __half2float(p.bias[gcol0 + i]) : 0.0f;
+          for (int i = 0; i < 16; ++i)
+            bi[i] = (gcol0 + i < p.N) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[gcol0 + i]) : 0.0f;
         }
         uint32_t packed[8];
         #pragma unroll
@@ -312,10 +309,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             y0 += __uint_as_float(fo[i]);
             y1 += __uint_as_float(fo[i + 1]);
           }
-          packed[i >> 1] = pack_half2(y0, y1);
+          packed[i >> 1] = Elem<TE>::pack2(y0, y1);
         }
         if (row_ok) {
-          __half* dst = p.Y + row * p.N + gcol0;
+          TE* dst = static_cast<TE*>(p.Y) + row * p.N + gcol0;
           #pragma unroll
           for (int g = 0; g < 2; ++g)
             if (gcol0 + g * 8 + 8 <= p.N)
@@ -378,8 +375,10 @@ int pair_kernel_max_clusters() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (g_max_pairs[dev] != 0) return g_max_pairs[dev];
-  if (cudaFuncSetAttribute(gemm_i8_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(gemm_i8_tc2_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(gemm_i8_tc2_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SMEM_BYTES) != cudaSuccess)
     return 0;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -393,7 +392,7 @@ int pair_kernel_max_clusters() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_i8_tc2_kernel, &cfg) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_i8_tc2_kernel<__half>, &cfg) != cudaSuccess) return 0;
   g_max_pairs[dev] = n;
   return n;
 }
@@ -406,10 +405,10 @@ cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s) {
   if (!make_map(&tmA, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K, a.T, a.K, BKB, BM)) return cudaErrorInvalidValue;
   if (!make_map(&tmB, a.CB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K, a.N, a.K, BKB, BN_HALF)) return cudaErrorInvalidValue;
   const bool outl = a.mode == 0 && a.n_out != nullptr && a.Xo != nullptr && a.Wo != nullptr;
+  const CUtensorMapDataType t16 = a.dtype == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   if (outl) {
-    if (!make_map(&tmAo, a.Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.ldo, a.T, a.ldo * 2, 64, BM))
-      return cudaErrorInvalidValue;
-    if (!make_map(&tmBo, a.Wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.ldo, a.N, a.ldo * 2, 64, BN_HALF))
+    if (!make_map(&tmAo, a.Xo, t16, a.ldo, a.T, a.ldo * 2, 64, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&tmBo, a.Wo, t16, a.ldo, a.N, a.ldo * 2, 64, BN_HALF))
       return cudaErrorInvalidValue;
   } else {
     tmAo = tmA;
@@ -448,7 +447,8 @@ cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_i8_tc2_kernel, tmA, tmB, tmAo, tmBo, p);
+  if (a.dtype == kBF16) return cudaLaunchKernelEx(&cfg, gemm_i8_tc2_kernel<__nv_bfloat16>, tmA, tmB, tmAo, tmBo, p);
+  return cudaLaunchKernelEx(&cfg, gemm_i8_tc2_kernel<__half>, tmA, tmB, tmAo, tmBo, p);
 }
 
 }  // namespace i8mp

@@ -15,8 +15,8 @@
 // token rows g and g+8; two MMAs consume them (bytes 0-7, then 8-15).  Every
 // thread issues the weight loads of two K-steps for all 4 row groups before
 // its first MMA, so 8 x 16 bytes per thread are in flight.
-// Epilogue: Y = fp16(acc * sA[t] * SCB[j] / 127^2 + sum_o Xo[t,o] * Wo[j,o] + b[j])
-// with Wo[j,o] = fp16((CB[j, idx[o]] * SCB[j]) / 127) recomputed from CB; the
+// Epilogue: Y = TE(acc * sA[t] * SCB[j] / 127^2 + sum_o Xo[t,o] * Wo[j,o] + b[j])
+// with Wo[j,o] = TE((CB[j, idx[o]] * SCB[j]) / 127) recomputed from CB; the
 // outlier operands of a 32-row chunk are staged in shared memory, 64 outlier
 // columns at a time.
 #include "kernels.h"
@@ -36,13 +36,13 @@ struct DvParams {
   const float* sA;
   const int8_t* CB;
   const float* SCB;
-  const __half* bias;
-  const __half* Xo;
+  const void* bias;  // TE[N] or null
+  const void* Xo;    // TE[T,ldo]
   int64_t ldo;
   const int32_t* idx;
   const int32_t* n_out;
-  const __half* Wf;  // fp16 weight (has_fp16_weights=True) or null
-  __half* Y;
+  const void* Wf;    // TE[N,K] 16-bit weight (has_fp16_weights=True) or null
+  void* Y;           // TE[T,N]
   int32_t* acc_out;
   int64_t T, N, K;
   int mode;
@@ -65,7 +65,9 @@ __device__ __forceinline__ uint4 ld_stream(const int8_t* p) {
   return v;
 }
 
+template <typename TE>
 __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvParams p) {
+  using E = Elem<TE>;
   __shared__ int32_t red[DV_WARPS][DV_RG][32][4];
   __shared__ float wo_s[DV_RG * 8][DV_OB + 1];
   __shared__ float xo_s[kDecodeMaxT][DV_OB + 1];
@@ -167,10 +169,10 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
         if (j < g_end * 8) {
           const int64_t col = __ldg(&p.idx[ob + o]);
           if (p.Wf != nullptr) {
-            wv = __half2float(p.Wf[j * p.K + col]);
+            wv = E::to_float(static_cast<const TE*>(p.Wf)[j * p.K + col]);
           } else {
             const float cbv = static_cast<float>(__ldg(&p.CB[j * p.K + col]));
-            wv = __half2float(__float2half_rn(__fdiv_rn(__fmul_rn(cbv, __ldg(&p.SCB[j])), 127.0f)));
+            wv = E::to_float(E::from_float(__fdiv_rn(__fmul_rn(cbv, __ldg(&p.SCB[j])), 127.0f)));
           }
         }
         wo_s[r][o] = wv;
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
       for (int e = threadIdx.x; e < kDecodeMaxT * nb; e += DV_THREADS) {
         const int t = e / nb;
         const int o = e - t * nb;
-        xo_s[t][o] = (t < p.T) ? __half2float(p.Xo[t * p.ldo + ob + o]) : 0.0f;
+        xo_s[t][o] = (t < p.T) ? E::to_float(static_cast<const TE*>(p.Xo)[t * p.ldo + ob + o]) : 0.0f;
       }
       __syncthreads();
       #pragma unroll
@@ -199,8 +201,8 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
       }
       const float scb = __ldg(&p.SCB[j]);
       float y = static_cast<float>(acc[h]) * (__ldg(&p.sA[tok[h]]) * (1.0f / 16129.0f) * scb) + yo[h];
-      if (p.bias != nullptr) y += __half2float(p.bias[j]);
-      p.Y[tok[h] * p.N + j] = __float2half_rn(y);
+      if (p.bias != nullptr) y += E::to_float(static_cast<const TE*>(p.bias)[j]);
+      static_cast<TE*>(p.Y)[tok[h] * p.N + j] = E::from_float(y);
     }
     __syncthreads();
   }
@@ -240,7 +242,8 @@ cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel, p);
+  if (a.dtype == kBF16) return cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel<__nv_bfloat16>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel<__half>, p);
 }
 
 }  // namespace i8mp

@@ -10,46 +10,51 @@
 
 namespace i8mp {
 
-// Weight quantisation: W fp16 [N,K] -> CB int8 [N,K], SCB fp32 [N].
-cudaError_t launch_quantize_weight(const __half* W, int64_t N, int64_t K, int8_t* CB, float* SCB,
+// Element type of the 16-bit operands (X, Xo, Wo, bias, Y, Wf): `dtype` is a
+// DType (kF16 or kBF16) throughout.
+
+// Weight quantisation: W [N,K] (16-bit) -> CB int8 [N,K], SCB fp32 [N].
+cudaError_t launch_quantize_weight(const void* W, int dtype, int64_t N, int64_t K, int8_t* CB, float* SCB,
                                    cudaStream_t s);
 
 // Column outlier mask (atomicOr into a zeroed mask) followed, in the last CTA
 // to finish, by compaction into the ascending idx list and n_out.
-// `hbits` is the largest fp16 magnitude bit pattern whose value is <= threshold.
-// Also writes prefix[w] = number of outlier columns in mask words 0..w-1.
-cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
+// `hbits` is the largest magnitude bit pattern of the element type whose value
+// is <= threshold.  Also writes prefix[w] = number of outlier columns in mask
+// words 0..w-1.
+cudaError_t launch_outliers(const void* X, int dtype, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
                             uint32_t* prefix, int32_t* idx, int32_t* n_out, DevStatus* st, cudaStream_t s);
 
-// Row-wise absmax int8 quantisation over non-outlier columns, fp16 gather of
+// Row-wise absmax int8 quantisation over non-outlier columns, 16-bit gather of
 // the outlier activation columns into Xo, and (when `with_wo`) the gather and
 // dequantisation of the matching weight columns into Wo -- or, when `Wf` (the
-// fp16 weight of a has_fp16_weights=True layer) is given, its own columns.
+// 16-bit weight of a has_fp16_weights=True layer) is given, its own columns.
 // `pdl`: launch with programmatic stream serialisation (only when the previous
 // operation in the stream is the outlier-pass kernel).
-cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_t* mask, const uint32_t* prefix,
-                            const int32_t* idx, const int32_t* n_out, int8_t* Xq, float* sA, __half* Xo,
-                            int64_t ldo, const int8_t* CB, const float* SCB, int64_t N, __half* Wo, bool with_wo,
-                            const __half* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s);
+cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, const uint32_t* mask,
+                            const uint32_t* prefix, const int32_t* idx, const int32_t* n_out, int8_t* Xq, float* sA,
+                            void* Xo, int64_t ldo, const int8_t* CB, const float* SCB, int64_t N, void* Wo,
+                            bool with_wo, const void* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s);
 
 struct GemmArgs {
   const int8_t* Xq;      // [T,K]
   const int8_t* CB;      // [N,K]
-  const __half* Xo;      // [T,ldo] (may be null when no outliers are possible)
-  const __half* Wo;      // [N,ldo]
+  const void* Xo;        // [T,ldo] 16-bit (may be null when no outliers are possible)
+  const void* Wo;        // [N,ldo] 16-bit
   int64_t ldo;
   const float* sA;       // [T]
   const float* SCB;      // [N]
-  const __half* bias;    // [N] or null
-  __half* Y;             // [T,N] fp16 output (mode 0)
+  const void* bias;      // [N] 16-bit, or null
+  void* Y;               // [T,N] 16-bit output (mode 0)
   int32_t* acc_out;      // [T,N] raw int32 accumulators (mode 1)
   const int32_t* n_out;  // device count of outlier columns, or null (= 0)
   const int32_t* idx;    // ascending outlier columns (decode path)
   DevStatus* st;
   int64_t T, N, K;
-  int mode;              // 0: fused fp16 Y, 1: int32 accumulators only
+  int mode;              // 0: fused 16-bit Y, 1: int32 accumulators only
   bool pdl = false;      // launch with programmatic stream serialisation (previous op is our kernel)
-  const __half* Wf = nullptr;  // fp16 weight [N,K] (has_fp16_weights=True): outlier weights come from it
+  const void* Wf = nullptr;  // 16-bit weight [N,K] (has_fp16_weights=True): outlier weights come from it
+  int dtype = kF16;          // element type of Xo, Wo, bias, Y, Wf
 };
 
 // Prefill: persistent tcgen05 kind::i8 GEMM with TMEM accumulators, fused

@@ -103,17 +103,16 @@ extern "C" i8_status int8_linear_forward_decode_static(const void* X, int64_t T,
   uint32_t* mask = reinterpret_cast<uint32_t*>(w + L.mask);
   float* sA = reinterpret_cast<float*>(w + L.sA);
   int8_t* Xq = reinterpret_cast<int8_t*>(w + L.Xq);
-  __half* Xo = reinterpret_cast<__half*>(w + L.Xo);
-  const __half* Xh = static_cast<const __half*>(X);
+  void* Xo = w + L.Xo;
 
   cudaError_t e;
   const uint32_t hb = int8_outlier_threshold_bits(threshold);
   if (hb == 0xffffffffu)
     e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
   else
-    e = launch_outliers(Xh, T, K, hb, mask, mask + (K + 31) / 32, idx, n_out, dst, stream);
+    e = launch_outliers(X, kF16, T, K, hb, mask, mask + (K + 31) / 32, idx, n_out, dst, stream);
   if (e != cudaSuccess) return I8_ERR_CUDA;
-  e = launch_rowquant(Xh, T, K, mask, mask + (K + 31) / 32, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, nullptr,
+  e = launch_rowquant(X, kF16, T, K, mask, mask + (K + 31) / 32, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, nullptr,
                       false, nullptr, num_sms, dst, hb != 0xffffffffu, stream);
   if (e != cudaSuccess) return I8_ERR_CUDA;
 
@@ -125,8 +124,8 @@ extern "C" i8_status int8_linear_forward_decode_static(const void* X, int64_t T,
   a.ldo = L.ldo;
   a.sA = sA;
   a.SCB = SCB;
-  a.bias = static_cast<const __half*>(bias);
-  a.Y = static_cast<__half*>(Y);
+  a.bias = bias;
+  a.Y = Y;
   a.acc_out = nullptr;
   a.n_out = n_out;
   a.idx = idx;

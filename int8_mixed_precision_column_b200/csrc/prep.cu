@@ -3,6 +3,8 @@
 //  * the column outlier mask and its compaction into the ascending index list;
 //  * row-wise absmax int8 quantisation of the non-outlier activations, and the
 //    gathers that feed the 16-bit outlier product.
+// Every kernel is a template over the 16-bit element type (fp16 or bf16; the
+// bitsandbytes Linear8bitLt docstring speaks of "fp16 / bf16 weights").
 //
 // Method: "Hugging Face integrates LLM.int8() 8-bit matrix multiplication into
 // Transformers and Accelerate", sections "Core idea of LLM.int8()" (steps 1-2)
@@ -17,8 +19,10 @@ namespace i8mp {
 // Weight quantisation: one warp per output row j.
 // SCB[j] = max_k |W[j,k]|; CB[j,k] = clamp(roundf(W[j,k] * (127/SCB[j])), +-127).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quantize_weight_kernel(const __half* __restrict__ W, int64_t N, int64_t K,
+template <typename TE>
+__global__ void __launch_bounds__(256) quantize_weight_kernel(const TE* __restrict__ W, int64_t N, int64_t K,
                                                               int8_t* __restrict__ CB, float* __restrict__ SCB) {
+  using E = Elem<TE>;
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= N) return;
@@ -27,9 +31,9 @@ __global__ void __launch_bounds__(256) quantize_weight_kernel(const __half* __re
   float m = 0.0f;
   for (int64_t i = lane; i < nv; i += 32) {
     uint4 v = __ldg(src + i);
-    const __half* h = reinterpret_cast<const __half*>(&v);
+    const TE* h = reinterpret_cast<const TE*>(&v);
     #pragma unroll
-    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(__half2float(h[e])));
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(E::to_float(h[e])));
   }
   m = warp_max(m);
   const float inv = scale_inv(m);
@@ -37,20 +41,25 @@ __global__ void __launch_bounds__(256) quantize_weight_kernel(const __half* __re
   uint2* dst = reinterpret_cast<uint2*>(CB + row * K);
   for (int64_t i = lane; i < nv; i += 32) {
     uint4 v = __ldg(src + i);
-    const __half* h = reinterpret_cast<const __half*>(&v);
+    const TE* h = reinterpret_cast<const TE*>(&v);
     uint32_t lo = 0, hi = 0;
     #pragma unroll
-    for (int e = 0; e < 4; ++e) lo |= (static_cast<uint32_t>(quant_code(__half2float(h[e]), inv)) & 0xffu) << (8 * e);
+    for (int e = 0; e < 4; ++e) lo |= (static_cast<uint32_t>(quant_code(E::to_float(h[e]), inv)) & 0xffu) << (8 * e);
     #pragma unroll
-    for (int e = 0; e < 4; ++e) hi |= (static_cast<uint32_t>(quant_code(__half2float(h[4 + e]), inv)) & 0xffu) << (8 * e);
+    for (int e = 0; e < 4; ++e)
+      hi |= (static_cast<uint32_t>(quant_code(E::to_float(h[4 + e]), inv)) & 0xffu) << (8 * e);
     dst[i] = make_uint2(lo, hi);
   }
 }
 
-cudaError_t launch_quantize_weight(const __half* W, int64_t N, int64_t K, int8_t* CB, float* SCB, cudaStream_t s) {
+cudaError_t launch_quantize_weight(const void* W, int dtype, int64_t N, int64_t K, int8_t* CB, float* SCB,
+                                   cudaStream_t s) {
   if (N == 0) return cudaSuccess;
-  const int64_t blocks = (N + 7) / 8;
-  quantize_weight_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(W, N, K, CB, SCB);
+  const unsigned blocks = static_cast<unsigned>((N + 7) / 8);
+  if (dtype == kBF16)
+    quantize_weight_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(W), N, K, CB, SCB);
+  else
+    quantize_weight_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), N, K, CB, SCB);
   return cudaGetLastError();
 }
 
@@ -59,56 +68,58 @@ cudaError_t launch_quantize_weight(const __half* W, int64_t N, int64_t K, int8_t
 //
 // Each thread owns 8 consecutive columns (one 16-byte load per row) and ORs
 // together, over its rows, the bits "|x| > threshold".  The comparison is done
-// on fp16 magnitude bit patterns: for non-NaN fp16 values the magnitude order
-// equals the order of the 15-bit patterns, so |x| > threshold  <=>
-// (bits & 0x7fff) > hbits, where hbits is the largest pattern whose value is
-// <= threshold (computed on the host).  NaN patterns (> 0x7c00) are excluded so
-// that NaN never flags a column.
+// on 16-bit magnitude bit patterns: for non-NaN fp16 or bf16 values the
+// magnitude order equals the order of the 15-bit patterns, so |x| > threshold
+// <=> (bits & 0x7fff) > hbits, where hbits is the largest pattern whose value
+// is <= threshold (computed on the host).  NaN patterns (above the infinity
+// pattern) are excluded so that NaN never flags a column.
 // CTA shape: `wc` of the 8 warps sit side by side along the columns (each warp
 // 256 columns = 512 contiguous bytes of a row), the other 8/wc split the rows;
 // the launcher uses wc = 1.  Four lanes' flag bytes make one mask word, ORed
-// into the mask with one atomicOr.  The last CTA to finish compacts the mask into the ascending
-// idx list and records, per mask word, how many outlier columns precede it
-// (prefix), so that the rank of an outlier column is prefix[w] + popc(lower
-// bits of word w).
+// into the mask with one atomicOr.  The last CTA to finish compacts the mask
+// into the ascending idx list and records, per mask word, how many outlier
+// columns precede it (prefix), so that the rank of an outlier column is
+// prefix[w] + popc(lower bits of word w).
 // ---------------------------------------------------------------------------
 constexpr int kMaskThreads = 256;
 constexpr int kMaskUnroll = 4;
 
-// Largest magnitude bit pattern among the 8 halves of v (fp16 max of |x|; max
-// ignores a NaN operand, so a NaN can only raise the result to a NaN pattern
-// when every element is NaN -- the caller then takes the exact path).
+// Largest magnitude bit pattern among the 8 elements of v (16-bit max of |x|;
+// max ignores a NaN operand, so a NaN can only raise the result to a NaN
+// pattern when every element is NaN -- the caller then takes the exact path).
+template <typename TE>
 __device__ __forceinline__ uint32_t chunk_max_mag(const uint4& v) {
-  const uint32_t w[4] = {v.x & 0x7fff7fffu, v.y & 0x7fff7fffu, v.z & 0x7fff7fffu, v.w & 0x7fff7fffu};
-  const __half2 m = __hmax2(__hmax2(*reinterpret_cast<const __half2*>(&w[0]), *reinterpret_cast<const __half2*>(&w[1])),
-                            __hmax2(*reinterpret_cast<const __half2*>(&w[2]), *reinterpret_cast<const __half2*>(&w[3])));
-  const uint32_t mm = *reinterpret_cast<const uint32_t*>(&m);
-  return max(mm & 0xffffu, mm >> 16);
+  using E = Elem<TE>;
+  const uint32_t m = E::max2(E::max2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu), E::max2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu));
+  return max(m & 0xffffu, m >> 16);
 }
 
 // Exact flags of one 8-column chunk; chunks whose largest magnitude is not
 // above the threshold (nearly all of them) are settled by chunk_max_mag alone.
+template <typename TE>
 __device__ __forceinline__ uint32_t flag_bits8(const uint4& v, uint32_t h2) {
-  if (chunk_max_mag(v) <= (h2 & 0xffffu)) return 0u;
+  if (chunk_max_mag<TE>(v) <= (h2 & 0xffffu)) return 0u;
+  const uint32_t inf2 = Elem<TE>::kInfBits | (Elem<TE>::kInfBits << 16);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t bits = 0;
   #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t a = w[i] & 0x7fff7fffu;
-    const uint32_t m = __vcmpgtu2(a, h2) & __vcmpleu2(a, 0x7c007c00u);
+    const uint32_t m = __vcmpgtu2(a, h2) & __vcmpleu2(a, inf2);
     bits |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * i);
   }
   return bits;
 }
 
-__global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const __half* __restrict__ X, int64_t T, int64_t K,
+template <typename TE>
+__global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const TE* __restrict__ X, int64_t T, int64_t K,
                                                                     uint32_t hbits, int wc, int64_t rows_per_cta,
                                                                     uint32_t* __restrict__ mask,
                                                                     uint32_t* __restrict__ prefix, int32_t* __restrict__ idx,
                                                                     int32_t* __restrict__ n_out, DevStatus* st) {
   __shared__ int s_last;
   __shared__ int s_scan[kMaskThreads];
-  griddep_launch_dependents();  // the row quantisation may start loading X meanwhile
+  griddep_launch_dependents();  // the row quantisation may start meanwhile
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int wcol = warp % wc;        // warp position along the columns
@@ -121,7 +132,7 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const __half
 
   uint32_t bits = 0;
   if (col8 < K) {
-    const __half* base = X + col8;
+    const TE* base = X + col8;
     int64_t r = r0 + wrow;
     #pragma unroll 1
     for (; r + (kMaskUnroll - 1) * wr < r1; r += kMaskUnroll * wr) {
@@ -129,10 +140,10 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const __half
       #pragma unroll
       for (int u = 0; u < kMaskUnroll; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(base + (r + u * wr) * K));
       #pragma unroll
-      for (int u = 0; u < kMaskUnroll; ++u) bits |= flag_bits8(v[u], h2);
+      for (int u = 0; u < kMaskUnroll; ++u) bits |= flag_bits8<TE>(v[u], h2);
     }
     #pragma unroll 1
-    for (; r < r1; r += wr) bits |= flag_bits8(__ldg(reinterpret_cast<const uint4*>(base + r * K)), h2);
+    for (; r < r1; r += wr) bits |= flag_bits8<TE>(__ldg(reinterpret_cast<const uint4*>(base + r * K)), h2);
   }
   // lanes 4i..4i+3 hold the 4 bytes of one mask word
   uint32_t word = bits << ((lane & 3) * 8);
@@ -182,7 +193,7 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const __half
   }
 }
 
-cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
+cudaError_t launch_outliers(const void* X, int dtype, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
                             uint32_t* prefix, int32_t* idx, int32_t* n_out, DevStatus* st, cudaStream_t s) {
   // The 8 warps split the rows (measured faster than warps side by side along
   // the columns, which gives fewer, longer-lived CTAs).
@@ -192,7 +203,12 @@ cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbit
   const int64_t chunks = (T + rows_per_cta - 1) / rows_per_cta;
   if (slabs > 0x7fffffff || chunks > 65535) return cudaErrorInvalidValue;
   dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(chunks));
-  outlier_mask_kernel<<<grid, kMaskThreads, 0, s>>>(X, T, K, hbits, wc, rows_per_cta, mask, prefix, idx, n_out, st);
+  if (dtype == kBF16)
+    outlier_mask_kernel<__nv_bfloat16><<<grid, kMaskThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(X), T, K, hbits,
+                                                                      wc, rows_per_cta, mask, prefix, idx, n_out, st);
+  else
+    outlier_mask_kernel<__half><<<grid, kMaskThreads, 0, s>>>(static_cast<const __half*>(X), T, K, hbits, wc,
+                                                              rows_per_cta, mask, prefix, idx, n_out, st);
   return cudaGetLastError();
 }
 
@@ -201,17 +217,18 @@ cudaError_t launch_outliers(const __half* X, int64_t T, int64_t K, uint32_t hbit
 //
 // Rows: one warp per token row t, two passes over the row (the second mostly
 // from L1/L2), with 8 independent 16-byte loads in flight per lane.
-//   pass 1: absmax over the non-outlier columns, kept as an fp16 magnitude bit
-//           pattern (integer max of (bits & 0x7fff) equals the magnitude max
-//           for finite values); chunks without outlier columns use an fp16 max
-//           of |x|; a warp shuffle reduces it -- no block barrier;
+//   pass 1: absmax over the non-outlier columns, kept as a 16-bit magnitude
+//           bit pattern (integer max of (bits & 0x7fff) equals the magnitude
+//           max for finite values); chunks without outlier columns use a
+//           16-bit max of |x|; a warp shuffle reduces it -- no block barrier;
 //   pass 2: codes clamp(round_half_away(x * fp32(127/absmax))) packed 8 per
 //           8-byte store, outlier values written to Xo[t, rank] straight from
 //           registers, rank = prefix[word] + popc(lower bits of the word).
-// Xo is zero-padded to the next multiple of 64 (the fp16 outlier K-block).
-// Wo blocks (blockIdx >= row blocks): Wo[j, o] = fp16((CB[j, idx[o]] * SCB[j]) / 127)
+// Xo is zero-padded to the next multiple of 64 (the 16-bit outlier K-block).
+// Wo blocks (blockIdx >= row blocks): Wo[j, o] = TE((CB[j, idx[o]] * SCB[j]) / 127)
 // with the same padding, four independent gathers per thread in flight (only
-// when the tensor-core product consumes Wo).
+// when the tensor-core product consumes Wo).  With a 16-bit weight Wf (the
+// has_fp16_weights=True layer) Wo[j, o] = Wf[j, idx[o]] instead.
 // ---------------------------------------------------------------------------
 constexpr int kRowThreads = 256;
 constexpr int kRowWarps = kRowThreads / 32;
@@ -223,8 +240,9 @@ __device__ __forceinline__ uint32_t mask_byte(const uint32_t* mask, int64_t chun
 }
 
 // Largest magnitude pattern among the non-outlier elements of a chunk.
+template <typename TE>
 __device__ __forceinline__ uint32_t chunk_max_mag_kept(const uint4& v, uint32_t mb) {
-  if (mb == 0) return chunk_max_mag(v);
+  if (mb == 0) return chunk_max_mag<TE>(v);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t m = 0;
   #pragma unroll
@@ -244,12 +262,13 @@ __device__ __forceinline__ int round_away_code(float y) {
   return (y < 0.0f) ? -q : q;
 }
 
+template <typename TE>
 __device__ __forceinline__ uint2 row_codes_fast(const uint4& v, uint32_t mb, float inv) {
-  const __half2* h = reinterpret_cast<const __half2*>(&v);
+  const uint32_t pairs[4] = {v.x, v.y, v.z, v.w};
   uint32_t w[2] = {0u, 0u};
   #pragma unroll
   for (int p = 0; p < 4; ++p) {
-    const float2 f = __half22float2(h[p]);
+    const float2 f = Elem<TE>::to_float2(pairs[p]);
     const int q0 = ((mb >> (2 * p)) & 1u) ? 0 : round_away_code(__fmul_rn(f.x, inv));
     const int q1 = ((mb >> (2 * p + 1)) & 1u) ? 0 : round_away_code(__fmul_rn(f.y, inv));
     w[p >> 1] |= ((static_cast<uint32_t>(q0) & 0xffu) | ((static_cast<uint32_t>(q1) & 0xffu) << 8)) << (16 * (p & 1));
@@ -258,9 +277,10 @@ __device__ __forceinline__ uint2 row_codes_fast(const uint4& v, uint32_t mb, flo
 }
 
 // Scatter the outlier entries of one 8-column chunk into the Xo row.
+template <typename TE>
 __device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, int64_t chunk, const uint32_t* mask,
-                                                 const uint32_t* prefix, __half* xo_row) {
-  const __half* h = reinterpret_cast<const __half*>(&v);
+                                                 const uint32_t* prefix, TE* xo_row) {
+  const TE* h = reinterpret_cast<const TE*>(&v);
   const uint32_t mw = __ldg(&mask[chunk >> 2]);
   const uint32_t base = __ldg(&prefix[chunk >> 2]);
   const int sh = static_cast<int>(chunk & 3) * 8;
@@ -269,12 +289,14 @@ __device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, in
     if ((mb >> e) & 1u) xo_row[base + __popc(mw & ((1u << (sh + e)) - 1u))] = h[e];
 }
 
+template <typename TE>
 __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
-    const __half* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
+    const TE* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
     const uint32_t* __restrict__ prefix, const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p,
-    int8_t* __restrict__ Xq, float* __restrict__ sA, __half* __restrict__ Xo, int64_t ldo,
-    const int8_t* __restrict__ CB, const float* __restrict__ SCB, int64_t N, __half* __restrict__ Wo,
-    const __half* __restrict__ Wf, int64_t row_blocks, int64_t wo_blocks) {
+    int8_t* __restrict__ Xq, float* __restrict__ sA, TE* __restrict__ Xo, int64_t ldo,
+    const int8_t* __restrict__ CB, const float* __restrict__ SCB, int64_t N, TE* __restrict__ Wo,
+    const TE* __restrict__ Wf, int64_t row_blocks, int64_t wo_blocks) {
+  using E = Elem<TE>;
   const int lane = threadIdx.x & 31;
   griddep_launch_dependents();
   griddep_wait();  // mask, prefix, idx, n_out come from the outlier pass
@@ -289,7 +311,7 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
     for (int64_t e0 = (static_cast<int64_t>(blockIdx.x) - row_blocks) * kRowThreads * kWoUnroll + threadIdx.x;
          e0 < total; e0 += stride) {
       int8_t cbv[kWoUnroll];
-      __half wfv[kWoUnroll];
+      TE wfv[kWoUnroll];
       int64_t jj[kWoUnroll], oo[kWoUnroll];
       #pragma unroll
       for (int u = 0; u < kWoUnroll; ++u) {
@@ -298,15 +320,15 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
         oo[u] = e - jj[u] * npad;
         const bool live = e < total && oo[u] < n_out;
         cbv[u] = (live && Wf == nullptr) ? __ldg(&CB[jj[u] * K + __ldg(&idx[oo[u]])]) : int8_t(0);
-        wfv[u] = (live && Wf != nullptr) ? Wf[jj[u] * K + __ldg(&idx[oo[u]])] : __float2half_rn(0.0f);
+        wfv[u] = (live && Wf != nullptr) ? Wf[jj[u] * K + __ldg(&idx[oo[u]])] : E::from_float(0.0f);
       }
       #pragma unroll
       for (int u = 0; u < kWoUnroll; ++u) {
         const int64_t e = e0 + static_cast<int64_t>(u) * kRowThreads;
         if (e < total) {
-          __half v = wfv[u];
+          TE v = wfv[u];
           if (oo[u] < n_out && Wf == nullptr)
-            v = __float2half_rn(__fdiv_rn(__fmul_rn(static_cast<float>(cbv[u]), __ldg(&SCB[jj[u]])), 127.0f));
+            v = E::from_float(__fdiv_rn(__fmul_rn(static_cast<float>(cbv[u]), __ldg(&SCB[jj[u]])), 127.0f));
           Wo[jj[u] * ldo + oo[u]] = v;
         }
       }
@@ -330,17 +352,17 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
     #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
       const int64_t c = c0 + 32 * u;
-      if (c < nv) mmax = max(mmax, chunk_max_mag_kept(v[u], mask_byte(mask, c)));
+      if (c < nv) mmax = max(mmax, chunk_max_mag_kept<TE>(v[u], mask_byte(mask, c)));
     }
   }
   #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
-  const float absmax = __half2float(__ushort_as_half(static_cast<unsigned short>(mmax)));
+  const float absmax = E::mag_to_float(mmax);
   const float inv = scale_inv(absmax);
   if (lane == 0) sA[t] = absmax;
 
   uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
-  __half* xo_row = Xo + t * ldo;
+  TE* xo_row = Xo + t * ldo;
   for (int64_t c0 = lane; c0 < nv; c0 += 32 * kRowUnroll) {
     uint4 v[kRowUnroll];
     #pragma unroll
@@ -353,18 +375,29 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
       const int64_t c = c0 + 32 * u;
       if (c < nv) {
         const uint32_t mb = mask_byte(mask, c);
-        dst[c] = row_codes_fast(v[u], mb, inv);
-        if (mb) scatter_outliers(v[u], mb, c, mask, prefix, xo_row);
+        dst[c] = row_codes_fast<TE>(v[u], mb, inv);
+        if (mb) scatter_outliers<TE>(v[u], mb, c, mask, prefix, xo_row);
       }
     }
   }
-  for (int64_t o = n_out + lane; o < npad; o += 32) xo_row[o] = __float2half_rn(0.0f);
+  for (int64_t o = n_out + lane; o < npad; o += 32) xo_row[o] = E::from_float(0.0f);
 }
 
-cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_t* mask, const uint32_t* prefix,
-                            const int32_t* idx, const int32_t* n_out, int8_t* Xq, float* sA, __half* Xo, int64_t ldo,
-                            const int8_t* CB, const float* SCB, int64_t N, __half* Wo, bool with_wo,
-                            const __half* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s) {
+template <typename TE>
+static cudaError_t launch_rowquant_t(const cudaLaunchConfig_t& cfg, const void* X, int64_t T, int64_t K,
+                                     const uint32_t* mask, const uint32_t* prefix, const int32_t* idx,
+                                     const int32_t* n_out, int8_t* Xq, float* sA, void* Xo, int64_t ldo,
+                                     const int8_t* CB, const float* SCB, int64_t N, void* Wo, const void* Wf,
+                                     int64_t row_blocks, int64_t wo_blocks) {
+  return cudaLaunchKernelEx(&cfg, rowquant_kernel<TE>, static_cast<const TE*>(X), T, K, mask, prefix, idx, n_out, Xq,
+                            sA, static_cast<TE*>(Xo), ldo, CB, SCB, N, static_cast<TE*>(Wo),
+                            static_cast<const TE*>(Wf), row_blocks, wo_blocks);
+}
+
+cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, const uint32_t* mask,
+                            const uint32_t* prefix, const int32_t* idx, const int32_t* n_out, int8_t* Xq, float* sA,
+                            void* Xo, int64_t ldo, const int8_t* CB, const float* SCB, int64_t N, void* Wo,
+                            bool with_wo, const void* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s) {
   (void)st;
   int64_t wo_blocks = 0;
   if (with_wo) {
@@ -386,8 +419,11 @@ cudaError_t launch_rowquant(const __half* X, int64_t T, int64_t K, const uint32_
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, rowquant_kernel, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N, Wo,
-                            Wf, row_blocks, wo_blocks);
+  if (dtype == kBF16)
+    return launch_rowquant_t<__nv_bfloat16>(cfg, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N, Wo,
+                                            Wf, row_blocks, wo_blocks);
+  return launch_rowquant_t<__half>(cfg, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N, Wo, Wf,
+                                   row_blocks, wo_blocks);
 }
 
 }  // namespace i8mp

@@ -24,6 +24,8 @@ STATUS_NAMES = {0: "I8_OK", 1: "I8_ERR_INVALID_ARG", 2: "I8_ERR_WORKSPACE", 3: "
 
 PATH_AUTO, PATH_TENSOR_CORE, PATH_DECODE, PATH_TENSOR_CORE_1SM = 0, 1, 2, 3
 DECODE_MAX_T = 16
+I8_DTYPE_F16, I8_DTYPE_BF16 = 0, 1
+_DTYPES = {torch.float16: I8_DTYPE_F16, torch.bfloat16: I8_DTYPE_BF16}
 
 _lib = None
 _lock = threading.Lock()
@@ -68,6 +70,11 @@ SIGNATURES = {
                                         ctypes.POINTER(ctypes.c_int)]),
     "int8_layer_unpack": (_I32, [_P, _SZ, _P, _P, _P]),
     "int8_linear_forward_decode_static": (_I32, [_P, _I64, _I64, _P, _P, _P, _I64, _F32, _P, _P, _P, _P]),
+    "int8_quantize_weight_ex": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P]),
+    "int8_linear_forward_ex": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _I64, _F32, _P, _P, _P, _P, _SZ, _I32,
+                                      ctypes.POINTER(ctypes.c_void_p), _P]),
+    "int8_linear_forward_fp16w_ex": (_I32, [_P, _I32, _I64, _I64, _P, _P, _I64, _F32, _P, _P, _P, _P, _SZ, _P]),
+    "int8_outlier_threshold_bits_ex": (ctypes.c_uint32, [_F32, _I32]),
 }
 
 
@@ -123,8 +130,16 @@ def int8_status_string(status: int) -> str:
     return lib().int8_status_string(status).decode()
 
 
-def int8_outlier_threshold_bits(threshold: float) -> int:
-    return int(lib().int8_outlier_threshold_bits(threshold))
+def _dtype_code(t: torch.Tensor, name: str) -> int:
+    if t.dtype not in _DTYPES:
+        raise ValueError(f"{name}: expected float16 or bfloat16, got {t.dtype}")
+    return _DTYPES[t.dtype]
+
+
+def int8_outlier_threshold_bits(threshold: float, dtype: torch.dtype = torch.float16) -> int:
+    if dtype == torch.float16:
+        return int(lib().int8_outlier_threshold_bits(threshold))
+    return int(lib().int8_outlier_threshold_bits_ex(threshold, _DTYPES[dtype]))
 
 
 def int8_linear_workspace_bytes(T: int, K: int, N: int) -> int:
@@ -139,14 +154,19 @@ def int8_linear_workspace_layout(T: int, K: int, N: int) -> dict:
 
 def int8_quantize_weight(W: torch.Tensor, CB: torch.Tensor | None = None, SCB: torch.Tensor | None = None,
                          stream=None):
-    """W fp16 [N,K] -> (CB int8 [N,K], SCB fp32 [N])."""
+    """W fp16 or bf16 [N,K] -> (CB int8 [N,K], SCB fp32 [N])."""
     N, K = W.shape
-    _require(W, torch.float16, (N, K), "W")
+    dt = _dtype_code(W, "W")
+    _require(W, W.dtype, (N, K), "W")
     CB = torch.empty((N, K), dtype=torch.int8, device=W.device) if CB is None else CB
     SCB = torch.empty((N,), dtype=torch.float32, device=W.device) if SCB is None else SCB
     _require(CB, torch.int8, (N, K), "CB")
     _require(SCB, torch.float32, (N,), "SCB")
-    _check("int8_quantize_weight", lib().int8_quantize_weight(_ptr(W), N, K, _ptr(CB), _ptr(SCB), _stream(stream)))
+    if dt == I8_DTYPE_F16:
+        st = lib().int8_quantize_weight(_ptr(W), N, K, _ptr(CB), _ptr(SCB), _stream(stream))
+    else:
+        st = lib().int8_quantize_weight_ex(_ptr(W), dt, N, K, _ptr(CB), _ptr(SCB), _stream(stream))
+    _check("int8_quantize_weight", st)
     return CB, SCB
 
 
@@ -160,23 +180,30 @@ def new_workspace(T: int, K: int, N: int, device="cuda") -> torch.Tensor:
 def int8_linear_forward(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor, bias: torch.Tensor | None,
                         threshold: float, *, Y=None, idx=None, n_out=None, workspace=None,
                         path: int = PATH_AUTO, stream=None):
-    """Returns (Y fp16 [T,N], idx int32 [K] (first n_out valid), n_out int32 [1], workspace)."""
+    """Returns (Y [T,N], idx int32 [K] (first n_out valid), n_out int32 [1], workspace).
+    X, bias and Y share one element type: fp16, or bf16 (the *_ex entry point)."""
     T, K = X.shape
     N = CB.shape[0]
-    _require(X, torch.float16, (T, K), "X")
+    dt = _dtype_code(X, "X")
+    _require(X, X.dtype, (T, K), "X")
     _require(CB, torch.int8, (N, K), "CB")
     _require(SCB, torch.float32, (N,), "SCB")
     if bias is not None:
-        _require(bias, torch.float16, (N,), "bias")
+        _require(bias, X.dtype, (N,), "bias")
     dev = X.device
-    Y = torch.empty((T, N), dtype=torch.float16, device=dev) if Y is None else Y
+    Y = torch.empty((T, N), dtype=X.dtype, device=dev) if Y is None else Y
     idx = torch.empty((K,), dtype=torch.int32, device=dev) if idx is None else idx
     n_out = torch.empty((1,), dtype=torch.int32, device=dev) if n_out is None else n_out
     workspace = new_workspace(T, K, N, dev) if workspace is None else workspace
-    _require(Y, torch.float16, (T, N), "Y")
-    st = lib().int8_linear_forward_path(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N, float(threshold),
-                                        _ptr(Y), _ptr(idx), _ptr(n_out), _ptr(workspace), workspace.numel(),
-                                        int(path), _stream(stream))
+    _require(Y, X.dtype, (T, N), "Y")
+    if dt == I8_DTYPE_F16:
+        st = lib().int8_linear_forward_path(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N, float(threshold),
+                                            _ptr(Y), _ptr(idx), _ptr(n_out), _ptr(workspace), workspace.numel(),
+                                            int(path), _stream(stream))
+    else:
+        st = lib().int8_linear_forward_ex(_ptr(X), dt, T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N, float(threshold),
+                                          _ptr(Y), _ptr(idx), _ptr(n_out), _ptr(workspace), workspace.numel(),
+                                          int(path), None, _stream(stream))
     _check("int8_linear_forward", st)
     return Y, idx, n_out, workspace
 
@@ -189,30 +216,43 @@ def int8_linear_forward_timed(X, CB, SCB, bias, threshold, Y, idx, n_out, worksp
     T, K = X.shape
     N = CB.shape[0]
     arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
-    st = lib().int8_linear_forward_timed(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N, float(threshold),
-                                         _ptr(Y), _ptr(idx), _ptr(n_out), _ptr(workspace), workspace.numel(),
-                                         int(path), arr, _stream(stream))
+    dt = _dtype_code(X, "X")
+    if dt == I8_DTYPE_F16:
+        st = lib().int8_linear_forward_timed(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N, float(threshold),
+                                             _ptr(Y), _ptr(idx), _ptr(n_out), _ptr(workspace), workspace.numel(),
+                                             int(path), arr, _stream(stream))
+    else:
+        st = lib().int8_linear_forward_ex(_ptr(X), dt, T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N, float(threshold),
+                                          _ptr(Y), _ptr(idx), _ptr(n_out), _ptr(workspace), workspace.numel(),
+                                          int(path), arr, _stream(stream))
     _check("int8_linear_forward_timed", st)
 
 
 def int8_linear_forward_fp16w(X: torch.Tensor, W: torch.Tensor, bias: torch.Tensor | None, threshold: float, *,
                               Y=None, idx=None, n_out=None, workspace=None, stream=None):
-    """has_fp16_weights=True forward: W fp16 [N,K] is quantised inside every call.
+    """has_fp16_weights=True forward: W [N,K] (fp16, or bf16 like X) is quantised inside every call.
     Returns (Y, idx, n_out, workspace); CB/SCB of this call sit in the workspace."""
     T, K = X.shape
     N = W.shape[0]
-    _require(X, torch.float16, (T, K), "X")
-    _require(W, torch.float16, (N, K), "W")
+    dt = _dtype_code(X, "X")
+    _require(X, X.dtype, (T, K), "X")
+    _require(W, X.dtype, (N, K), "W")
     if bias is not None:
-        _require(bias, torch.float16, (N,), "bias")
+        _require(bias, X.dtype, (N,), "bias")
     dev = X.device
-    Y = torch.empty((T, N), dtype=torch.float16, device=dev) if Y is None else Y
+    Y = torch.empty((T, N), dtype=X.dtype, device=dev) if Y is None else Y
     idx = torch.empty((K,), dtype=torch.int32, device=dev) if idx is None else idx
     n_out = torch.empty((1,), dtype=torch.int32, device=dev) if n_out is None else n_out
     if workspace is None:
         workspace = torch.empty(int(lib().int8_linear_fp16w_workspace_bytes(T, K, N)), dtype=torch.uint8, device=dev)
-    st = lib().int8_linear_forward_fp16w(_ptr(X), T, K, _ptr(W), _ptr(bias), N, float(threshold), _ptr(Y), _ptr(idx),
-                                         _ptr(n_out), _ptr(workspace), workspace.numel(), _stream(stream))
+    if dt == I8_DTYPE_F16:
+        st = lib().int8_linear_forward_fp16w(_ptr(X), T, K, _ptr(W), _ptr(bias), N, float(threshold), _ptr(Y),
+                                             _ptr(idx), _ptr(n_out), _ptr(workspace), workspace.numel(),
+                                             _stream(stream))
+    else:
+        st = lib().int8_linear_forward_fp16w_ex(_ptr(X), dt, T, K, _ptr(W), _ptr(bias), N, float(threshold),
+                                                _ptr(Y), _ptr(idx), _ptr(n_out), _ptr(workspace), workspace.numel(),
+                                                _stream(stream))
     _check("int8_linear_forward_fp16w", st)
     return Y, idx, n_out, workspace
 
@@ -255,8 +295,9 @@ def int8_linear_forward_host(X_host: torch.Tensor, CB: torch.Tensor, SCB: torch.
     _check("int8_linear_forward_host", st)
 
 
-def workspace_views(workspace: torch.Tensor, T: int, K: int, N: int) -> dict:
-    """Typed views of the forward's intermediate buffers inside ``workspace``."""
+def workspace_views(workspace: torch.Tensor, T: int, K: int, N: int, dtype: torch.dtype = torch.float16) -> dict:
+    """Typed views of the forward's intermediate buffers inside ``workspace``
+    (``dtype``: the forward's 16-bit element type, that of Xo and Wo)."""
     L = int8_linear_workspace_layout(T, K, N)
     ldo = L["ldo"]
     nw = (K + 31) // 32
@@ -268,8 +309,8 @@ def workspace_views(workspace: torch.Tensor, T: int, K: int, N: int) -> dict:
         "mask": view(L["mask"], nw * 4, torch.int32, (nw,)),
         "sA": view(L["sA"], T * 4, torch.float32, (T,)),
         "Xq": view(L["Xq"], T * K, torch.int8, (T, K)),
-        "Xo": view(L["Xo"], T * ldo * 2, torch.float16, (T, ldo)),
-        "Wo": view(L["Wo"], N * ldo * 2, torch.float16, (N, ldo)),
+        "Xo": view(L["Xo"], T * ldo * 2, dtype, (T, ldo)),
+        "Wo": view(L["Wo"], N * ldo * 2, dtype, (N, ldo)),
         "ldo": ldo,
     }
 

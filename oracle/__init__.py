@@ -13,6 +13,12 @@ from .llm_int8 import (  # noqa: F401
     int8_matmul,
     linear_forward,
     linear_forward_fp16w,
+    bf16_to_f32,
+    f32_to_bf16,
+    quantize_weight_bf16,
+    linear_forward_bf16,
+    linear_forward_fp16w_bf16,
+    y_tolerance_bf16,
     outlier_index,
     outlier_mask,
     outlier_operands,

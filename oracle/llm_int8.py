@@ -236,6 +236,86 @@ def linear_forward_fp16w(X, W, bias, threshold, rows=None) -> dict:
             "Xo": Xo, "Wo": Wo, "acc": acc, "Y": Y}
 
 
+# ---------------------------------------------------------------------------
+# bf16 (the module is documented for "fp16 / bf16 weights"): numpy has no
+# bfloat16 type, so bf16 values are carried as uint16 bit patterns -- the
+# upper half of the fp32 pattern.
+# ---------------------------------------------------------------------------
+
+def bf16_to_f32(u16: np.ndarray) -> np.ndarray:
+    """Exact widening: the bf16 pattern is the top 16 bits of the fp32 pattern."""
+    return (np.asarray(u16, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 pattern, round to nearest, ties to even (NaN stays NaN)."""
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    rounded = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    nan = np.isnan(np.asarray(x, dtype=np.float32))
+    return np.where(nan, np.uint16(0x7FC0), rounded).astype(np.uint16)
+
+
+def quantize_weight_bf16(W_u16: np.ndarray):
+    """bf16 W [N,K] (patterns) -> (CB, SCB): the absmax rule of quantize_weight."""
+    Wf = bf16_to_f32(W_u16)
+    SCB = np.abs(Wf).max(axis=1).astype(np.float32) if Wf.shape[1] else np.zeros(Wf.shape[0], np.float32)
+    return absmax_codes(Wf, SCB), SCB
+
+
+def linear_forward_bf16(X_u16, CB, SCB, bias_u16, threshold, rows=None) -> dict:
+    """The forward for bf16 activations / bias / output; outlier weights are
+    bf16((CB * SCB) / 127).  Every step is the fp16 forward's step with bf16
+    in place of fp16."""
+    Xf = bf16_to_f32(X_u16)
+    thr = np.float32(threshold)
+    K = Xf.shape[1]
+    mask = (np.abs(Xf) > thr).any(axis=0) if (thr > 0 and Xf.shape[0]) else np.zeros(K, bool)
+    idx = outlier_index(mask)
+    Xs = Xf if rows is None else Xf[np.asarray(rows)]
+    kept = np.where(mask[None, :], np.float32(0.0), np.abs(Xs)).astype(np.float32)
+    sA = kept.max(axis=1).astype(np.float32) if K else np.zeros(Xs.shape[0], np.float32)
+    Xq = absmax_codes(np.where(mask[None, :], np.float32(0.0), Xs), sA)
+    Xq[:, mask] = 0
+    Xo = Xs[:, idx]                                                   # exact (bf16 values)
+    Wo = bf16_to_f32(f32_to_bf16(dequantize_weight(CB[:, idx], SCB)))
+    acc = int8_matmul(Xq, CB)
+    bias = None if bias_u16 is None else bf16_to_f32(bias_u16)
+    Y = acc.astype(np.float64) * sA.astype(np.float64)[:, None] * SCB.astype(np.float64)[None, :]
+    Y = Y / float(Q_MAX * Q_MAX)
+    if idx.size:
+        Y = Y + Xo.astype(np.float64) @ Wo.astype(np.float64).T
+    if bias is not None:
+        Y = Y + bias.astype(np.float64)[None, :]
+    return {"mask": mask, "idx": idx, "n_out": int(idx.size), "Xq": Xq, "sA": sA, "Xo": f32_to_bf16(Xo),
+            "Wo": f32_to_bf16(Wo), "acc": acc, "Y": Y}
+
+
+def linear_forward_fp16w_bf16(X_u16, W_u16, bias_u16, threshold, rows=None) -> dict:
+    """has_fp16_weights=True with bf16 operands: W (bf16 patterns) is quantised
+    in the forward, and the outlier columns are multiplied with W's own bf16
+    columns W[:, idx] (the reading of linear_forward_fp16w, with bf16 in place
+    of fp16)."""
+    CB, SCB = quantize_weight_bf16(W_u16)
+    r = linear_forward_bf16(X_u16, CB, SCB, None, threshold, rows)
+    idx = r["idx"]
+    Wo = bf16_to_f32(np.asarray(W_u16, dtype=np.uint16)[:, idx]).astype(np.float64)
+    Xo = bf16_to_f32(r["Xo"]).astype(np.float64)
+    Y = r["acc"].astype(np.float64) * r["sA"].astype(np.float64)[:, None] * SCB.astype(np.float64)[None, :]
+    Y = Y / float(Q_MAX * Q_MAX)
+    if idx.size:
+        Y = Y + Xo @ Wo.T
+    if bias_u16 is not None:
+        Y = Y + bf16_to_f32(bias_u16).astype(np.float64)[None, :]
+    r.update({"CB": CB, "SCB": SCB, "Wo": np.asarray(W_u16, dtype=np.uint16)[:, idx], "Y": Y})
+    return r
+
+
+def y_tolerance_bf16(Yref: np.ndarray) -> float:
+    """Allowed max |Y - Yref| for a bf16 output: the output rounding alone
+    can reach 2^-9 |Y| (8 stored mantissa bits), so 2^-8 * max|Yref| + 2e-3."""
+    return 2.0**-8 * float(np.abs(Yref).max(initial=0.0)) + 2e-3
+
+
 def y_tolerance(Yref: np.ndarray) -> float:
     """Allowed max |Y - Yref| for the fp16 output: 1e-3 * max|Yref| + 2e-3."""
     return 1e-3 * float(np.abs(Yref).max(initial=0.0)) + 2e-3

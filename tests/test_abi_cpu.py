@@ -113,3 +113,39 @@ def test_small_workspace_rejected(lib):
     fake = ctypes.c_void_p(1 << 20)
     st = lib.int8_linear_forward(fake, 4, 64, fake, fake, None, 64, 6.0, fake, fake, fake, fake, 16, None)
     assert st == 2  # I8_ERR_WORKSPACE
+
+
+def _bf16_values():
+    bits = np.arange(0, 0x10000, dtype=np.uint32)
+    return bits, (bits << 16).view(np.float32)
+
+
+@pytest.mark.parametrize("thr", [6.0, 0.1, 1e-8, 3.14159, 6.000001, 6.03125, 3.0e38, 3.4e38, float("inf"), 1e-40])
+def test_bf16_threshold_bits_match_fp32_comparison(lib, thr):
+    """bf16: (bits & 0x7fff) > H and not NaN  <=>  |float(x)| > float32(thr), for every bf16 x."""
+    H = native.int8_outlier_threshold_bits(thr, native.torch.bfloat16)
+    bits, vals = _bf16_values()
+    mag = bits & 0x7FFF
+    kernel_rule = (mag > H) & (mag <= 0x7F80)
+    with np.errstate(invalid="ignore"):
+        fp32_rule = np.abs(vals) > np.float32(thr)
+    assert np.array_equal(kernel_rule, fp32_rule)
+
+
+@pytest.mark.parametrize("thr", [0.0, -1.0, float("nan")])
+def test_bf16_threshold_off(lib, thr):
+    assert lib.int8_outlier_threshold_bits_ex(thr, native.I8_DTYPE_BF16) == 0xFFFFFFFF
+
+
+def test_unknown_dtype_rejected_before_any_cuda_call(lib):
+    assert lib.int8_outlier_threshold_bits_ex(6.0, 2) == 0xFFFFFFFE
+    fake = ctypes.c_void_p(1 << 20)
+    big = native.int8_linear_workspace_bytes(4, 64, 64)
+    for dt in (-1, 2, 7):
+        st = lib.int8_linear_forward_ex(fake, dt, 4, 64, fake, fake, None, 64, 6.0, fake, fake, fake, fake, big, 0,
+                                        None, None)
+        assert st == 1
+        assert lib.int8_quantize_weight_ex(fake, dt, 64, 64, fake, fake, None) == 1
+        st = lib.int8_linear_forward_fp16w_ex(fake, dt, 4, 64, fake, None, 64, 6.0, fake, fake, fake, fake, 1 << 30,
+                                              None)
+        assert st == 1

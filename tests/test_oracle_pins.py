@@ -336,6 +336,89 @@ def check_fp16w_outlier_weights_are_the_fp16_columns():
     np.testing.assert_allclose(r["Y"], exact, rtol=0, atol=1e-9)
 
 
+def check_bf16_conversions():
+    """Widening is exact; narrowing picks the nearest bf16, ties to the even pattern."""
+    pats = np.arange(0, 0x10000, dtype=np.uint32).astype(np.uint16)
+    f = O.bf16_to_f32(pats)
+    ok = ~np.isnan(f)
+    assert np.array_equal(O.f32_to_bf16(f[ok]), pats[ok])
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.normal(0, 10, 20000), rng.normal(0, 1e-30, 2000)]).astype(np.float32)
+    mid = (O.bf16_to_f32(pats[:0x7F80].astype(np.uint16)).astype(np.float64))  # non-negative finite
+    b = O.f32_to_bf16(x)
+    got = O.bf16_to_f32(b).astype(np.float64)
+    ax = np.abs(x.astype(np.float64))
+    lo_i = np.clip(np.searchsorted(mid, ax, side="right") - 1, 0, mid.size - 2)
+    lo, hi = mid[lo_i], mid[lo_i + 1]
+    best = np.where(ax - lo < hi - ax, lo, np.where(ax - lo > hi - ax, hi, np.where(lo_i % 2 == 0, lo, hi)))
+    assert np.array_equal(np.abs(got), best)
+
+
+def check_bf16_worked_example(read_golden):
+    g = read_golden("absmax_worked_example.txt")
+    v = O.f32_to_bf16(np.array([float(t) for t in g["vector"]], np.float32))
+    CB, SCB = O.quantize_weight_bf16(v[None, :])
+    assert abs(127.0 / float(SCB[0]) - float(g["scale_printed"][0])) <= float(g["scale_printed_tolerance"][0])
+    assert CB[0].tolist() == [int(t) for t in g["codes_derived"]]
+
+
+def check_bf16_lossless_closed_form():
+    for with_out in (False, True):
+        X, W, b, cols = lossless_problem(31 + with_out, with_out)   # integers: exact in bf16 too
+        Xb, Wb, bb = (O.f32_to_bf16(a.astype(np.float32)) for a in (X, W, b))
+        CB, SCB = O.quantize_weight_bf16(Wb)
+        r = O.linear_forward_bf16(Xb, CB, SCB, bb, 150.0 if with_out else 0.0)
+        assert r["idx"].tolist() == cols
+        # outlier magnitudes up to 400 are not all bf16 integers: use the bf16 values
+        Xv, Wv, bv = (O.bf16_to_f32(a).astype(np.float64) for a in (Xb, Wb, bb))
+        exact = Xv @ Wv.T + bv
+        assert np.array_equal(r["Y"], exact)
+
+
+def check_bf16_all_columns_flagged():
+    rng = np.random.default_rng(8)
+    X = O.f32_to_bf16(rng.choice([-1.0, 1.0], (6, 32)).astype(np.float32) * rng.uniform(0.2, 3, (6, 32)).astype(np.float32))
+    W = O.f32_to_bf16(rng.normal(0, 0.05, (16, 32)).astype(np.float32))
+    CB, SCB = O.quantize_weight_bf16(W)
+    r = O.linear_forward_bf16(X, CB, SCB, None, 0.1)
+    assert r["n_out"] == 32 and np.all(r["acc"] == 0)
+    Wdq = np.empty(CB.shape, np.float32)
+    for j in range(CB.shape[0]):
+        for k in range(CB.shape[1]):
+            Wdq[j, k] = np.float32(np.float32(CB[j, k]) * SCB[j]) / np.float32(127)
+    want = O.bf16_to_f32(X).astype(np.float64) @ O.bf16_to_f32(O.f32_to_bf16(Wdq)).astype(np.float64).T
+    np.testing.assert_allclose(r["Y"], want, rtol=1e-12, atol=1e-12)
+
+
+def check_bf16_fp16w_all_columns_is_exact_product():
+    """bf16 has_fp16_weights=True with every column an outlier: Y = X W^T + bias
+    over the bf16 values, exactly (the int8 part is all zero)."""
+    rng = np.random.default_rng(9)
+    X = O.f32_to_bf16(rng.choice([-1.0, 1.0], (5, 48)).astype(np.float32) * rng.uniform(0.5, 4, (5, 48)).astype(np.float32))
+    W = O.f32_to_bf16(rng.normal(0, 0.05, (32, 48)).astype(np.float32))
+    b = O.f32_to_bf16(rng.normal(0, 0.1, 32).astype(np.float32))
+    r = O.linear_forward_fp16w_bf16(X, W, b, 0.25)
+    assert r["n_out"] == 48 and np.all(r["acc"] == 0) and np.array_equal(r["Wo"], W)
+    want = np.empty((5, 32))
+    for t in range(5):
+        for j in range(32):
+            want[t, j] = sum(float(O.bf16_to_f32(X[t, k])) * float(O.bf16_to_f32(W[j, k])) for k in range(48))
+            want[t, j] += float(O.bf16_to_f32(b[j]))
+    np.testing.assert_allclose(r["Y"], want, rtol=1e-12, atol=1e-12)
+
+
+def check_bf16_fp16w_without_outliers_is_int8_forward():
+    """With the decomposition off, the bf16 weight only enters through CB/SCB."""
+    rng = np.random.default_rng(10)
+    X = O.f32_to_bf16(rng.normal(0, 1, (7, 64)).astype(np.float32))
+    W = O.f32_to_bf16(rng.normal(0, 0.02, (48, 64)).astype(np.float32))
+    r = O.linear_forward_fp16w_bf16(X, W, None, 0.0)
+    CB, SCB = O.quantize_weight_bf16(W)
+    q = O.linear_forward_bf16(X, CB, SCB, None, 0.0)
+    assert r["n_out"] == 0 and np.array_equal(r["CB"], CB)
+    np.testing.assert_array_equal(r["Y"], q["Y"])
+
+
 ALL_PINS = [
     check_worked_example, check_rounding, check_range_and_absmax, check_recovery_half_step,
     check_mask_bruteforce, check_toy_columns, check_issue_1609, check_threshold_off,
@@ -344,6 +427,9 @@ ALL_PINS = [
     check_bias_linearity, check_error_bound, check_outlier_operands,
     check_fp16w_all_columns_is_exact_product, check_fp16w_without_outliers_equals_int8_forward,
     check_fp16w_outlier_weights_are_the_fp16_columns,
+    check_bf16_conversions, check_bf16_worked_example, check_bf16_lossless_closed_form,
+    check_bf16_all_columns_flagged, check_bf16_fp16w_all_columns_is_exact_product,
+    check_bf16_fp16w_without_outliers_is_int8_forward,
 ]
 
 
