@@ -214,6 +214,158 @@ class ClockSampler:
 # our implementation
 # ---------------------------------------------------------------------------
 
+def run_sharded(args, rank, world, local_rank) -> dict | None:
+    """One layer split along N over the ranks (strong scaling: the total work
+    is the one layer), Y assembled on every rank by the product kernels'
+    stores into every rank's symmetric output buffer."""
+    from int8_mixed_precision_column_b200 import build, native, sharded
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build.build()
+    native.lib()
+    p = WORKLOADS[args.workload]("cuda", rank_seed(0))  # the same layer and batch on every rank
+    if args.threshold is not None:
+        p.threshold = args.threshold
+    T, K, N = p.T, p.K, p.N
+    CB, SCB = native.int8_quantize_weight(p.W)
+    del p.W
+    layer = sharded.NShardedLinear(CB, SCB, p.bias, T_max=T, mode="peer")
+    del CB, SCB
+    torch.cuda.empty_cache()
+    X = p.X
+    for _ in range(args.warmup):
+        layer.forward(X, p.threshold)
+    torch.cuda.synchronize()
+    st, where = layer.check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {native.int8_status_string(st)} at {where:#x}")
+    sampler = ClockSampler(pci_bus_id(dev))
+    if rank == 0:
+        sampler.start()
+        time.sleep(1.0)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.mark_begin()
+    e0.record()
+    for _ in range(args.steps):
+        layer.forward(X, p.threshold)
+    e1.record()
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    barrier(world)
+    clocks = sampler.stop() if rank == 0 else None
+    st, where = layer.check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {native.int8_status_string(st)} at {where:#x}")
+    ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
+    n_outliers = int(layer.n_out.item())
+    if rank != 0:
+        return None
+    ops = 2.0 * T * N * K
+    peaks, peak_src = load_peaks()
+    per_rank_ops = ops / world
+    achieved = per_rank_ops / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    return {
+        "metric": METRIC, "value": ops / (ms * 1e-3) / 1e12, "unit": "TOPS", "tokens_per_s": T / (ms * 1e-3),
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "int8 x int8 -> int32 (+ fp16 outlier product, fp32 accumulate), fp16 in/out",
+        "data": "synthetic (seeded; X ~ N(0,1) with planted outlier columns, W ~ N(0, 0.02^2))",
+        "config": {"workload": args.workload, "T": T, "K": K, "N": N, "threshold": p.threshold,
+                   "n_out": n_outliers, "parallelism": f"N-sharded x{world}, Y gathered by peer stores",
+                   "l2": "inputs larger than L2 (no flush)" if T * K * 3 + N * K // world > 2 * L2_BYTES
+                   else "L2 not flushed (working set below 2 x L2)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS", "frac": achieved / peak,
+                     "traffic": None, "traffic_source": "whole sharded forward per rank (3 kernels + 2 barriers)",
+                     "kernel": "whole forward", "peak_source": f"{peak_src} bf16_tflops (burst) x {INT8_PER_BF16}"},
+        "gpu_launches": (3 if p.threshold > 0 else 2) * args.steps,
+        "clocks": clocks, "e2e": None, "device": torch.cuda.get_device_name(dev),
+    }
+
+
+def run_e2e(args, X, CB, SCB, bias, threshold, T, K, N, world, dev) -> dict:
+    """The metric end to end through the library's host-buffer calls.
+
+    Every step copies its X from pinned host memory, runs the forward and
+    copies Y, idx and n_out back.  Two forms: the blocking call
+    (int8_linear_forward_host, one step at a time) and the non-blocking one
+    (int8_linear_forward_host_async) alternating between two streams and two
+    workspaces, so one step's Y download overlaps the next step's X upload
+    and kernels.  The pipelined form is the reported value.
+    """
+    from int8_mixed_precision_column_b200 import native
+
+    Xh = X.cpu().pin_memory()
+    nbytes = native.int8_linear_forward_host_workspace_bytes(T, K, N)
+    slots = []
+    for _ in range(2):
+        slots.append({"stream": torch.cuda.Stream(dev),
+                      "ws": torch.empty(nbytes, dtype=torch.uint8, device=dev),
+                      "Y": torch.empty((T, N), dtype=X.dtype).pin_memory(),
+                      "idx": torch.empty((K,), dtype=torch.int32).pin_memory(),
+                      "n": torch.empty((1,), dtype=torch.int32).pin_memory()})
+    ne = max(3, min(args.steps, 20))
+    s0 = slots[0]
+
+    def blocking():
+        native.int8_linear_forward_host(Xh, CB, SCB, bias, threshold, s0["Y"], s0["ws"], s0["idx"], s0["n"])
+
+    for _ in range(min(args.warmup, 3)):
+        blocking()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(ne):
+        blocking()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    blocking_ms = reduce_max(e0.elapsed_time(e1) / ne, world, dev)
+
+    main = torch.cuda.current_stream(dev)
+
+    def pipelined(n):
+        start, ends = torch.cuda.Event(enable_timing=True), []
+        start.record(main)
+        for sl in slots:
+            sl["stream"].wait_event(start)
+        for i in range(n):
+            sl = slots[i % 2]
+            native.int8_linear_forward_host_async(Xh, CB, SCB, bias, threshold, sl["Y"], sl["ws"], sl["idx"],
+                                                  sl["n"], stream=sl["stream"])
+        for sl in slots:
+            ev = torch.cuda.Event()
+            ev.record(sl["stream"])
+            main.wait_event(ev)
+        end = torch.cuda.Event(enable_timing=True)
+        end.record(main)
+        return start, end
+
+    pipelined(min(args.warmup, 3) + 1)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = pipelined(ne)
+    torch.cuda.synchronize()
+    barrier(world)
+    for sl in slots:
+        st, where = native.int8_check_status(sl["ws"])
+        if st != 0:
+            raise RuntimeError(f"device status {native.int8_status_string(st)} at {where:#x}")
+    e2e_ms = reduce_max(start.elapsed_time(end) / ne, world, dev)
+    return {"value": whole_job(2.0 * T * N * K, T, world, e2e_ms)[0], "unit": "TOPS",
+            "ms_per_step": e2e_ms, "steps": ne,
+            "h2d_bytes_per_step": T * K * 2,
+            "d2h_bytes_per_step": T * N * 2 + K * 4 + 4,
+            "api": "int8_linear_forward_host_async on 2 streams (pinned host X/Y, resident CB/SCB)",
+            "blocking": {"value": whole_job(2.0 * T * N * K, T, world, blocking_ms)[0], "ms_per_step": blocking_ms,
+                         "api": "int8_linear_forward_host (one step at a time)"}}
+
+
 def run_ours(args, rank, world, local_rank) -> dict | None:
     from int8_mixed_precision_column_b200 import build, native
 
@@ -293,34 +445,12 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     total_ms = outer[0].elapsed_time(outer[1]) if not flush else sum(step_ms)
     ms_per_step = reduce_max(total_ms / nsteps, world, dev)
 
-    # end to end through the host-buffer entry point: pinned X in, Y/idx/n_out out, per step
+    # end to end through the host-buffer entry points: pinned X in, Y/idx/n_out out, every step
     e2e = None
-    if not args.no_e2e and elem == torch.float16:  # the host-buffer entry point takes fp16
-        Xh = X.cpu().pin_memory()
-        Yh = torch.empty((T, N), dtype=torch.float16).pin_memory()
-        idx_h = torch.empty((K,), dtype=torch.int32).pin_memory()
-        n_h = torch.empty((1,), dtype=torch.int32).pin_memory()
+    if not args.no_e2e and elem == torch.float16:  # the blocking host entry point takes fp16
         del ws
         torch.cuda.empty_cache()
-        wsh = torch.empty(native.int8_linear_forward_host_workspace_bytes(T, K, N), dtype=torch.uint8, device=dev)
-        for _ in range(min(args.warmup, 3)):
-            native.int8_linear_forward_host(Xh, CB, SCB, bias, p.threshold, Yh, wsh, idx_h, n_h)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ne = max(3, min(nsteps, 20))
-        barrier(world)
-        torch.cuda.synchronize()
-        e0.record()
-        for _ in range(ne):
-            native.int8_linear_forward_host(Xh, CB, SCB, bias, p.threshold, Yh, wsh, idx_h, n_h)
-        e1.record()
-        torch.cuda.synchronize()
-        barrier(world)
-        e2e_ms = reduce_max(e0.elapsed_time(e1) / ne, world, dev)
-        e2e = {"value": whole_job(2.0 * T * N * K, T, world, e2e_ms)[0], "unit": "TOPS",
-               "ms_per_step": e2e_ms, "steps": ne,
-               "h2d_bytes_per_step": T * K * 2,
-               "d2h_bytes_per_step": T * N * 2 + K * 4 + 4 + 64,
-               "api": "int8_linear_forward_host (pinned host X/Y, resident CB/SCB)"}
+        e2e = run_e2e(args, X, CB, SCB, bias, p.threshold, T, K, N, world, dev)
 
     if rank != 0:
         return None
@@ -478,6 +608,8 @@ def main() -> None:
                     help="product kernel: 0 auto, 1 tensor core (SM pairs), 2 decode GEMV, 3 tensor core (single SM)")
     ap.add_argument("--dtype", default="fp16", choices=["fp16", "bf16"],
                     help="16-bit element type of X, bias, Y and the outlier product")
+    ap.add_argument("--shard-n", action="store_true",
+                    help="split one layer along N over the ranks (strong scaling; Y gathered by peer stores)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -490,18 +622,27 @@ def main() -> None:
         if out is not None:
             print(json.dumps(out), flush=True)
         return
-    if world > 1:
+    pg = world > 1 or args.shard_n
+    if pg:
         import datetime
+        import socket
         import torch.distributed as dist
+        if world == 1:
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                os.environ.setdefault("MASTER_PORT", str(sk.getsockname()[1]))
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        out = run_ours(args, rank, world, local_rank)
+        out = run_sharded(args, rank, world, local_rank) if args.shard_n else run_ours(args, rank, world, local_rank)
         if out is not None:
             print(json.dumps(out), flush=True)
     finally:
-        if world > 1:
+        if pg:
             import torch.distributed as dist
             dist.destroy_process_group()
 

@@ -164,6 +164,19 @@ i8_status int8_linear_forward_host(const void* X_host, int64_t T, int64_t K, con
                                    int32_t* idx_host, int32_t* n_out_host, void* workspace,
                                    size_t workspace_bytes, cudaStream_t stream);
 
+/* As int8_linear_forward_host for element type `dtype` (I8_DTYPE_F16 or
+ * I8_DTYPE_BF16 below), but non-blocking: the copies and kernels are enqueued
+ * on `stream` and the call returns at once.  X_host, Y_host, idx_host and
+ * n_out_host must stay valid (and Y_host unread) until `stream` has been
+ * synchronised; then int8_check_status(workspace, ...) reads the status word.
+ * X_host and Y_host must be page-locked: pageable memory makes the copies
+ * synchronous.  Two calls on two streams with two workspaces overlap one
+ * forward's Y download with the next one's X upload and kernels. */
+i8_status int8_linear_forward_host_async(const void* X_host, int dtype, int64_t T, int64_t K, const int8_t* CB,
+                                         const float* SCB, const void* bias, int64_t N, float threshold,
+                                         void* Y_host, int32_t* idx_host, int32_t* n_out_host, void* workspace,
+                                         size_t workspace_bytes, cudaStream_t stream);
+
 /* As int8_linear_forward_path, and records caller-created CUDA events
  * (cudaEvent_t, passed as void*) on `stream` around the stages:
  * events[0] before the first stage, events[1] after the outlier pass,
@@ -279,6 +292,40 @@ i8_status int8_linear_forward_fp16w_ex(const void* X, int dtype, int64_t T, int6
                                        const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
                                        int32_t* n_out, void* workspace, size_t workspace_bytes,
                                        cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * N-sharded forward (one shard of the output features per GPU).
+ *
+ * The Hugging Face integration page ("Speed trade-offs", the table of
+ * BLOOM-176B runs) serves the INT8 model over several GPUs.  The forward
+ * splits along N with no exchange in the compute: every GPU holds the rows
+ * [col_offset, col_offset + N) of CB, SCB and bias, sees the whole X, finds
+ * the same outlier columns and row scales, and produces the matching column
+ * block of Y.  This call computes that block and stores it straight into up
+ * to 8 copies of the full output -- the caller's own and, for the gather, the
+ * same buffer of every other GPU mapped into this device's address space --
+ * so that the all-gather of Y happens inside the product kernel's epilogue.
+ *   X, dtype, T, K, threshold, idx, n_out, workspace, path: as
+ *             int8_linear_forward_ex (workspace sized for T, K, N).
+ *   CB, SCB, bias  this GPU's shard: [N,K], [N], [N] (bias may be NULL).
+ *   Y_dst     HOST array of n_dst (1..8) device pointers, each the start
+ *             (column 0) of a row-major [T, ldY] output of element type
+ *             `dtype`, 16-byte aligned; Y_dst[0] is this GPU's own.
+ *   ldY       row stride of every Y_dst in elements: a multiple of 8, >= N.
+ *   col_offset first column of this shard in Y: a multiple of 8, with
+ *             col_offset + N <= ldY.
+ * Columns outside [col_offset, col_offset + N) are not touched.  The stores to
+ * other GPUs' memory are complete when the kernel is; before any GPU reads
+ * its full Y, every GPU's forward must have completed (for example a
+ * stream-ordered barrier across the GPUs after this call).  Errors as
+ * int8_linear_forward_ex; a bad Y_dst, ldY or col_offset is
+ * I8_ERR_INVALID_ARG.
+ * ------------------------------------------------------------------------- */
+i8_status int8_linear_forward_sharded(const void* X, int dtype, int64_t T, int64_t K, const int8_t* CB,
+                                      const float* SCB, const void* bias, int64_t N, float threshold,
+                                      void* const* Y_dst, int n_dst, int64_t ldY, int64_t col_offset,
+                                      int32_t* idx, int32_t* n_out, void* workspace, size_t workspace_bytes,
+                                      int path, cudaStream_t stream);
 
 /* int8_outlier_threshold_bits for element type `dtype`: the largest magnitude
  * pattern of that type (bf16: 0..0x7f80) whose value is <= threshold.

@@ -130,7 +130,7 @@ cudaError_t launch_product(const GemmArgs& a, int path, bool gemv, int num_sms, 
 i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB, const void* bias,
                        int64_t N, float threshold, void* Y, int32_t* idx, int32_t* n_out, void* ws, size_t ws_bytes,
                        int path, void* const* events, cudaStream_t stream, int dtype = kF16,
-                       const void* Wf = nullptr) {
+                       const void* Wf = nullptr, int64_t ldY = 0, void* const* ydst = nullptr, int n_ydst = 0) {
   if (!shape_ok(T, K, N) || !dtype_ok(dtype)) return I8_ERR_INVALID_ARG;
   if (path < kPathAuto || path > kPathTensorCoreSingleSM) return I8_ERR_INVALID_ARG;
   if (path == kPathDecode && T > kDecodeMaxT) return I8_ERR_INVALID_ARG;
@@ -204,6 +204,9 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   a.pdl = true;  // follows the row quantisation kernel
   a.Wf = Wf;
   a.dtype = dtype;
+  a.ldY = ldY;
+  a.n_ydst = n_ydst;
+  for (int d = 0; d < n_ydst; ++d) a.ydst[d] = ydst[d];
   e = launch_product(a, path, gemv, num_sms, stream);
   if (e != cudaSuccess || !mark(3)) return I8_ERR_CUDA;
   return I8_OK;
@@ -299,6 +302,23 @@ i8_status int8_linear_forward_ex(const void* X, int dtype, int64_t T, int64_t K,
                       stream, dtype);
 }
 
+i8_status int8_linear_forward_sharded(const void* X, int dtype, int64_t T, int64_t K, const int8_t* CB,
+                                      const float* SCB, const void* bias, int64_t N, float threshold,
+                                      void* const* Y_dst, int n_dst, int64_t ldY, int64_t col_offset, int32_t* idx,
+                                      int32_t* n_out, void* workspace, size_t workspace_bytes, int path,
+                                      cudaStream_t stream) {
+  if (Y_dst == nullptr || n_dst < 1 || n_dst > kMaxYDst + 1) return I8_ERR_INVALID_ARG;
+  if (ldY < N || ldY % 8 != 0 || col_offset < 0 || col_offset % 8 != 0 || col_offset + N > ldY)
+    return I8_ERR_INVALID_ARG;
+  void* dst[kMaxYDst + 1];
+  for (int d = 0; d < n_dst; ++d) {
+    if (Y_dst[d] == nullptr || !aligned(Y_dst[d], 16)) return I8_ERR_INVALID_ARG;
+    dst[d] = static_cast<uint8_t*>(Y_dst[d]) + col_offset * 2;
+  }
+  return forward_impl(X, T, K, CB, SCB, bias, N, threshold, dst[0], idx, n_out, workspace, workspace_bytes, path,
+                      nullptr, stream, dtype, nullptr, ldY, dst + 1, n_dst - 1);
+}
+
 i8_status int8_check_status(void* workspace, uint32_t* where, cudaStream_t stream) {
   if (workspace == nullptr || !aligned(workspace, 256)) return I8_ERR_WORKSPACE;
   if (where != nullptr) *where = 0xffffffffu;  // "the synchronisation itself failed"
@@ -357,11 +377,12 @@ size_t int8_linear_forward_host_workspace_bytes(int64_t T, int64_t K, int64_t N)
   return static_cast<size_t>(make_host_extra(T, K, N).total);
 }
 
-i8_status int8_linear_forward_host(const void* X_host, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
-                                   const void* bias, int64_t N, float threshold, void* Y_host, int32_t* idx_host,
-                                   int32_t* n_out_host, void* workspace, size_t workspace_bytes,
-                                   cudaStream_t stream) {
-  if (!shape_ok(T, K, N)) return I8_ERR_INVALID_ARG;
+// The forward on host buffers: X in, forward, Y (and idx, n_out) out, all
+// enqueued on `stream`; `sync` waits and reads the status word.
+static i8_status host_forward(const void* X_host, int dtype, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                       const void* bias, int64_t N, float threshold, void* Y_host, int32_t* idx_host,
+                       int32_t* n_out_host, void* workspace, size_t workspace_bytes, cudaStream_t stream, bool sync) {
+  if (!shape_ok(T, K, N) || !dtype_ok(dtype)) return I8_ERR_INVALID_ARG;
   if (T > 0 && (X_host == nullptr || Y_host == nullptr)) return I8_ERR_INVALID_ARG;
   const HostExtra H = make_host_extra(T, K, N);
   const int8_ws_layout L = make_layout(T, K, N);
@@ -375,8 +396,8 @@ i8_status int8_linear_forward_host(const void* X_host, int64_t T, int64_t K, con
   const size_t ybytes = static_cast<size_t>(T) * N * 2;
   if (xbytes && cudaMemcpyAsync(Xd, X_host, xbytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return I8_ERR_CUDA;
-  i8_status st =
-      forward_impl(Xd, T, K, CB, SCB, bias, N, threshold, Yd, idxd, nd, workspace, L.total, 0, nullptr, stream);
+  i8_status st = forward_impl(Xd, T, K, CB, SCB, bias, N, threshold, Yd, idxd, nd, workspace, L.total, 0, nullptr,
+                              stream, dtype);
   if (st != I8_OK) return st;
   if (ybytes && cudaMemcpyAsync(Y_host, Yd, ybytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return I8_ERR_CUDA;
@@ -385,7 +406,23 @@ i8_status int8_linear_forward_host(const void* X_host, int64_t T, int64_t K, con
     return I8_ERR_CUDA;
   if (n_out_host && cudaMemcpyAsync(n_out_host, nd, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return I8_ERR_CUDA;
-  return int8_check_status(workspace, nullptr, stream);
+  return sync ? int8_check_status(workspace, nullptr, stream) : I8_OK;
+}
+
+i8_status int8_linear_forward_host(const void* X_host, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                                   const void* bias, int64_t N, float threshold, void* Y_host, int32_t* idx_host,
+                                   int32_t* n_out_host, void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
+  return host_forward(X_host, kF16, T, K, CB, SCB, bias, N, threshold, Y_host, idx_host, n_out_host, workspace,
+                      workspace_bytes, stream, true);
+}
+
+i8_status int8_linear_forward_host_async(const void* X_host, int dtype, int64_t T, int64_t K, const int8_t* CB,
+                                         const float* SCB, const void* bias, int64_t N, float threshold,
+                                         void* Y_host, int32_t* idx_host, int32_t* n_out_host, void* workspace,
+                                         size_t workspace_bytes, cudaStream_t stream) {
+  return host_forward(X_host, dtype, T, K, CB, SCB, bias, N, threshold, Y_host, idx_host, n_out_host, workspace,
+                      workspace_bytes, stream, false);
 }
 
 i8_status int8_gemm_i32(const int8_t* Xq, int64_t T, int64_t K, const int8_t* CB, int64_t N, int32_t* acc, int path,

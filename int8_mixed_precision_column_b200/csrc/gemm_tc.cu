@@ -56,6 +56,7 @@ struct Params {
   const void* bias;  // TE[N] or null
   void* Y;           // TE[T,N]
   int32_t* acc_out;
+  YDst yd;           // row stride of Y and its extra destinations
   const int32_t* n_out;
   DevStatus* st;
   int mode;
@@ -273,12 +274,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           packed[i >> 1] = Elem<TE>::pack2(y0, y1);
         }
         if (row_ok) {
-          TE* dst = static_cast<TE*>(p.Y) + row * p.N + gcol0;
+          const int64_t off = row * p.yd.ld + gcol0;
+          TE* dst = static_cast<TE*>(p.Y) + off;
           #pragma unroll
           for (int g = 0; g < 4; ++g)
-            if (gcol0 + g * 8 + 8 <= p.N)
-              reinterpret_cast<uint4*>(dst)[g] =
-                  make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+            if (gcol0 + g * 8 + 8 <= p.N) {
+              const uint4 v = make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+              reinterpret_cast<uint4*>(dst)[g] = v;
+              if (p.yd.n > 0) store_extra_u4<TE>(p.yd, off + g * 8, v);
+            }
         }
       }
       tc_fence_before();
@@ -369,6 +373,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t s) {
   p.bias = a.bias;
   p.Y = a.Y;
   p.acc_out = a.acc_out;
+  p.yd = make_ydst(a);
   p.n_out = outl ? a.n_out : nullptr;
   p.st = a.st;
   p.mode = a.mode;

@@ -44,6 +44,7 @@ struct DvParams {
   const void* Wf;    // TE[N,K] 16-bit weight (has_fp16_weights=True) or null
   void* Y;           // TE[T,N]
   int32_t* acc_out;
+  YDst yd;           // row stride of Y and its extra destinations
   int64_t T, N, K;
   int mode;
 };
@@ -65,7 +66,9 @@ __device__ __forceinline__ uint4 ld_stream(const int8_t* p) {
   return v;
 }
 
-template <typename TE>
+// kExtra: Y also goes to the extra destinations of p.yd (a separate
+// instantiation, so the single-destination kernel is not burdened by it).
+template <typename TE, bool kExtra>
 __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvParams p) {
   using E = Elem<TE>;
   __shared__ int32_t red[DV_WARPS][DV_RG][32][4];
@@ -202,7 +205,10 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
       const float scb = __ldg(&p.SCB[j]);
       float y = static_cast<float>(acc[h]) * (__ldg(&p.sA[tok[h]]) * (1.0f / 16129.0f) * scb) + yo[h];
       if (p.bias != nullptr) y += E::to_float(static_cast<const TE*>(p.bias)[j]);
-      static_cast<TE*>(p.Y)[tok[h] * p.N + j] = E::from_float(y);
+      const int64_t off = tok[h] * p.yd.ld + j;
+      const TE v = E::from_float(y);
+      static_cast<TE*>(p.Y)[off] = v;
+      if constexpr (kExtra) store_extra<TE>(p.yd, off, v);
     }
     __syncthreads();
   }
@@ -226,6 +232,7 @@ cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s) {
   p.Wf = a.Wf;
   p.Y = a.Y;
   p.acc_out = a.acc_out;
+  p.yd = make_ydst(a);
   p.T = a.T;
   p.N = a.N;
   p.K = a.K;
@@ -242,8 +249,12 @@ cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 1 : 0;
-  if (a.dtype == kBF16) return cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel<__nv_bfloat16>, p);
-  return cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel<__half>, p);
+  const bool extra = p.yd.n > 0;
+  if (a.dtype == kBF16)
+    return extra ? cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel<__nv_bfloat16, true>, p)
+                 : cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel<__nv_bfloat16, false>, p);
+  return extra ? cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel<__half, true>, p)
+               : cudaLaunchKernelEx(&cfg, gemv_i8_decode_kernel<__half, false>, p);
 }
 
 }  // namespace i8mp

@@ -36,6 +36,33 @@ cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, cons
                             void* Xo, int64_t ldo, const int8_t* CB, const float* SCB, int64_t N, void* Wo,
                             bool with_wo, const void* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s);
 
+// Extra destinations of Y besides `Y` itself: the same [T, ldY] buffer on the
+// other GPUs of an N-sharded layer (peer-mapped), so that one kernel computes
+// its column block and stores it everywhere.
+constexpr int kMaxYDst = 7;
+
+// Kernel-side view of the output layout: row stride and extra destinations.
+struct YDst {
+  int64_t ld;          // row stride of Y in elements
+  int n;               // number of extra destinations (0..kMaxYDst)
+  void* p[kMaxYDst];
+};
+
+// Store one 16-byte vector at element offset `off` of every extra destination
+// (the loop is unrolled so every index is a constant).
+template <typename TE>
+__device__ __forceinline__ void store_extra_u4(const YDst& y, int64_t off, const uint4& v) {
+  #pragma unroll
+  for (int d = 0; d < kMaxYDst; ++d)
+    if (d < y.n) *reinterpret_cast<uint4*>(static_cast<TE*>(y.p[d]) + off) = v;
+}
+template <typename TE>
+__device__ __forceinline__ void store_extra(const YDst& y, int64_t off, TE v) {
+  #pragma unroll
+  for (int d = 0; d < kMaxYDst; ++d)
+    if (d < y.n) static_cast<TE*>(y.p[d])[off] = v;
+}
+
 struct GemmArgs {
   const int8_t* Xq;      // [T,K]
   const int8_t* CB;      // [N,K]
@@ -55,7 +82,18 @@ struct GemmArgs {
   bool pdl = false;      // launch with programmatic stream serialisation (previous op is our kernel)
   const void* Wf = nullptr;  // 16-bit weight [N,K] (has_fp16_weights=True): outlier weights come from it
   int dtype = kF16;          // element type of Xo, Wo, bias, Y, Wf
+  int64_t ldY = 0;           // row stride of Y (and of every ydst) in elements; 0 means N
+  int n_ydst = 0;            // number of extra destinations in ydst (0..kMaxYDst)
+  void* ydst[kMaxYDst] = {};  // extra copies of Y (mode 0 only), same layout and column offset
 };
+
+inline YDst make_ydst(const GemmArgs& a) {
+  YDst y;
+  y.ld = a.ldY > 0 ? a.ldY : a.N;
+  y.n = a.n_ydst;
+  for (int d = 0; d < kMaxYDst; ++d) y.p[d] = d < a.n_ydst ? a.ydst[d] : nullptr;
+  return y;
+}
 
 // Prefill: persistent tcgen05 kind::i8 GEMM with TMEM accumulators, fused
 // kind::f16 outlier product and dequant/bias epilogue.

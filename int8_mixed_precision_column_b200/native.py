@@ -75,7 +75,13 @@ SIGNATURES = {
                                       ctypes.POINTER(ctypes.c_void_p), _P]),
     "int8_linear_forward_fp16w_ex": (_I32, [_P, _I32, _I64, _I64, _P, _P, _I64, _F32, _P, _P, _P, _P, _SZ, _P]),
     "int8_outlier_threshold_bits_ex": (ctypes.c_uint32, [_F32, _I32]),
+    "int8_linear_forward_sharded": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _I64, _F32,
+                                           ctypes.POINTER(ctypes.c_void_p), _I32, _I64, _I64, _P, _P, _P, _SZ,
+                                           _I32, _P]),
+    "int8_linear_forward_host_async": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _I64, _F32, _P, _P, _P, _P, _SZ,
+                                              _P]),
 }
+MAX_Y_DST = 8
 
 
 def lib() -> ctypes.CDLL:
@@ -257,6 +263,41 @@ def int8_linear_forward_fp16w(X: torch.Tensor, W: torch.Tensor, bias: torch.Tens
     return Y, idx, n_out, workspace
 
 
+def int8_linear_forward_sharded(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor, bias: torch.Tensor | None,
+                                threshold: float, Y_dst: list, ldY: int, col_offset: int, *, idx=None, n_out=None,
+                                workspace=None, path: int = PATH_AUTO, stream=None):
+    """One output-feature shard of the forward, stored into every buffer of
+    ``Y_dst`` (device pointers as ints, or tensors; [T, ldY] of X's dtype) at
+    columns [col_offset, col_offset + N).  Returns (idx, n_out, workspace)."""
+    T, K = X.shape
+    N = CB.shape[0]
+    dt = _dtype_code(X, "X")
+    _require(X, X.dtype, (T, K), "X")
+    _require(CB, torch.int8, (N, K), "CB")
+    _require(SCB, torch.float32, (N,), "SCB")
+    if bias is not None:
+        _require(bias, X.dtype, (N,), "bias")
+    if not 1 <= len(Y_dst) <= MAX_Y_DST:
+        raise ValueError(f"Y_dst: 1..{MAX_Y_DST} destinations, got {len(Y_dst)}")
+    ptrs = []
+    for y in Y_dst:
+        if isinstance(y, torch.Tensor):
+            _require(y, X.dtype, (T, ldY), "Y_dst[i]")
+            ptrs.append(y.data_ptr())
+        else:
+            ptrs.append(int(y))
+    dev = X.device
+    idx = torch.empty((K,), dtype=torch.int32, device=dev) if idx is None else idx
+    n_out = torch.empty((1,), dtype=torch.int32, device=dev) if n_out is None else n_out
+    workspace = new_workspace(T, K, N, dev) if workspace is None else workspace
+    arr = (ctypes.c_void_p * len(ptrs))(*[ctypes.c_void_p(q) for q in ptrs])
+    st = lib().int8_linear_forward_sharded(_ptr(X), dt, T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N, float(threshold),
+                                           arr, len(ptrs), int(ldY), int(col_offset), _ptr(idx), _ptr(n_out),
+                                           _ptr(workspace), workspace.numel(), int(path), _stream(stream))
+    _check("int8_linear_forward_sharded", st)
+    return idx, n_out, workspace
+
+
 def int8_check_status(workspace: torch.Tensor, stream=None) -> tuple[int, int]:
     where = ctypes.c_uint32(0)
     st = lib().int8_check_status(_ptr(workspace), ctypes.byref(where), _stream(stream))
@@ -293,6 +334,26 @@ def int8_linear_forward_host(X_host: torch.Tensor, CB: torch.Tensor, SCB: torch.
                                         _ptr(Y_host), _ptr(idx_host), _ptr(n_out_host), _ptr(workspace),
                                         workspace.numel(), _stream(stream))
     _check("int8_linear_forward_host", st)
+
+
+def int8_linear_forward_host_async(X_host: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor, bias, threshold: float,
+                                   Y_host: torch.Tensor, workspace: torch.Tensor, idx_host=None, n_out_host=None,
+                                   stream=None) -> None:
+    """Non-blocking forward on pinned host X/Y; synchronise ``stream``, then
+    call int8_check_status(workspace) before reading Y_host."""
+    T, K = X_host.shape
+    N = CB.shape[0]
+    dt = _dtype_code(X_host, "X_host")
+    if X_host.is_cuda or Y_host.is_cuda or Y_host.dtype != X_host.dtype:
+        raise ValueError("X_host/Y_host must be host tensors of one 16-bit dtype")
+    if not (X_host.is_pinned() and Y_host.is_pinned()):
+        raise ValueError("X_host/Y_host must be pinned (page-locked)")
+    if not (X_host.is_contiguous() and Y_host.is_contiguous()) or tuple(Y_host.shape) != (T, N):
+        raise ValueError("X_host/Y_host must be contiguous with shapes [T,K], [T,N]")
+    st = lib().int8_linear_forward_host_async(_ptr(X_host), dt, T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
+                                              float(threshold), _ptr(Y_host), _ptr(idx_host), _ptr(n_out_host),
+                                              _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("int8_linear_forward_host_async", st)
 
 
 def workspace_views(workspace: torch.Tensor, T: int, K: int, N: int, dtype: torch.dtype = torch.float16) -> dict:

@@ -323,6 +323,42 @@ def test_host_buffer_forward_matches_device_forward():
     assert torch.equal(Yh, g["Y"].cpu())
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_async_host_forward_on_two_streams(dtype):
+    """Non-blocking host-buffer forwards alternating on two streams and two
+    workspaces (the pipelined e2e form) give the device forward's outputs."""
+    p = workloads.llama7b_prefill(seed=2)
+    X = p.X.to(dtype)
+    W = p.W.to(dtype).cuda()
+    b = p.bias.to(dtype).cuda()
+    CB, SCB = native.int8_quantize_weight(W)
+    Y_ref, idx_ref, n_ref, _ = native.int8_linear_forward(X.cuda(), CB, SCB, b, p.threshold)
+    n = int(n_ref.item())
+    Xh = X.clone().pin_memory()
+    nbytes = native.int8_linear_forward_host_workspace_bytes(p.T, p.K, p.N)
+    slots = [(torch.cuda.Stream(), torch.empty(nbytes, dtype=torch.uint8, device="cuda"),
+              torch.empty((p.T, p.N), dtype=dtype).pin_memory(), torch.empty((p.K,), dtype=torch.int32).pin_memory(),
+              torch.empty((1,), dtype=torch.int32).pin_memory()) for _ in range(2)]
+    for i in range(5):
+        s, ws, Yh, idx_h, n_h = slots[i % 2]
+        native.int8_linear_forward_host_async(Xh, CB, SCB, b, p.threshold, Yh, ws, idx_h, n_h, stream=s)
+    torch.cuda.synchronize()
+    for s, ws, Yh, idx_h, n_h in slots:
+        assert native.int8_check_status(ws)[0] == 0
+        assert int(n_h) == n and torch.equal(idx_h[:n], idx_ref[:n].cpu())
+        assert torch.equal(Yh.view(torch.int16), Y_ref.cpu().view(torch.int16))
+
+
+def test_async_host_forward_rejects_pageable_buffers():
+    p = workloads.toy(seed=0)
+    CB, SCB = native.int8_quantize_weight(p.W.cuda())
+    ws = torch.empty(native.int8_linear_forward_host_workspace_bytes(p.T, p.K, p.N), dtype=torch.uint8,
+                     device="cuda")
+    with pytest.raises(ValueError):
+        native.int8_linear_forward_host_async(p.X, CB, SCB, None, 6.0, torch.empty((p.T, p.N), dtype=torch.float16),
+                                              ws)
+
+
 # ---------------------------------------------------------------------------
 # rounding and subnormal edge cases of the row codes and the outlier test
 # ---------------------------------------------------------------------------
