@@ -398,19 +398,26 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     scrub = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
 
     nsteps = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nsteps + args.warmup)]
+    # Steps are timed as plain forwards (the kernels chain by programmatic
+    # launch); the per-stage breakdown and the product kernel's duration come
+    # from a separate pass of int8_linear_forward_timed, whose stage events
+    # sit between the kernels.
+    nstage = max(3, min(nsteps, 20))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nstage)]
     for row in ev:
         for e in row:
             e.record()
+    bounds = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(nsteps)]
     outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
 
-    def step(i):
-        native.int8_linear_forward_timed(X, CB, SCB, bias, p.threshold, Y, idx, n_out, ws, ev[i], path=args.path)
+    def step():
+        native.int8_linear_forward(X, CB, SCB, bias, p.threshold, Y=Y, idx=idx, n_out=n_out, workspace=ws,
+                                   path=args.path)
 
     for i in range(args.warmup):
         if flush:
             scrub.add_(1)
-        step(nsteps + i)
+        step()
     torch.cuda.synchronize()
     st, where = native.int8_check_status(ws)
     if st != 0:
@@ -428,22 +435,32 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     for i in range(nsteps):
         if flush:
             scrub.add_(1)
-        step(i)
+        bounds[i][0].record()
+        step()
+        bounds[i][1].record()
     outer[1].record()
     torch.cuda.synchronize()
     sampler.mark_end()
     barrier(world)
     clocks = sampler.stop() if rank == 0 else None
-
     st, where = native.int8_check_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {native.int8_status_string(st)} at {where:#x}")
-    step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(nsteps)]
-    prod_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(nsteps)]
-    outl_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(nsteps)]
-    rowq_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(nsteps)]
+    step_ms = [bounds[i][0].elapsed_time(bounds[i][1]) for i in range(nsteps)]
     total_ms = outer[0].elapsed_time(outer[1]) if not flush else sum(step_ms)
     ms_per_step = reduce_max(total_ms / nsteps, world, dev)
+
+    for i in range(nstage):
+        if flush:
+            scrub.add_(1)
+        native.int8_linear_forward_timed(X, CB, SCB, bias, p.threshold, Y, idx, n_out, ws, ev[i], path=args.path)
+    torch.cuda.synchronize()
+    st, where = native.int8_check_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {native.int8_status_string(st)} at {where:#x}")
+    prod_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(nstage)]
+    outl_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(nstage)]
+    rowq_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(nstage)]
 
     # end to end through the host-buffer entry points: pinned X in, Y/idx/n_out out, every step
     e2e = None
@@ -498,6 +515,8 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
                    "elem": args.dtype,
                    "n_out": n_outliers, "parallelism": f"independent problem per rank x{world}",
                    "l2": "L2 flushed between steps" if flush else "inputs larger than L2 (no flush)"},
+        "stage_ms_note": "per-stage CUDA events from a separate pass with events between the kernels "
+                         "(no programmatic overlap there); value and ms_per_step time plain forwards",
         "stage_ms": {"outliers": statistics.mean(outl_ms), "rowquant": statistics.mean(rowq_ms),
                      "product": prod_avg},
         "roofline": roof,

@@ -181,7 +181,10 @@ i8_status int8_linear_forward_host_async(const void* X_host, int dtype, int64_t 
  * (cudaEvent_t, passed as void*) on `stream` around the stages:
  * events[0] before the first stage, events[1] after the outlier pass,
  * events[2] after the row quantisation, events[3] after the product kernel.
- * For measurement: event deltas time each kernel on its launching stream. */
+ * On the decode path (the weight-streaming product, T <= 16) the outlier pass
+ * and the row quantisation are one kernel: events[1] and events[2] both
+ * follow it.  For measurement: event deltas time each kernel on its launching
+ * stream (the events between kernels stop them from overlapping). */
 i8_status int8_linear_forward_timed(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
                                     const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
                                     int32_t* n_out, void* workspace, size_t workspace_bytes, int path,

@@ -153,8 +153,11 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   if (!mark(0)) return I8_ERR_CUDA;
   uint8_t* w = static_cast<uint8_t*>(ws);
   const uint64_t mask_bytes = static_cast<uint64_t>((K + 31) / 32) * 4;
-  // status word + mask start at zero for every forward
-  cudaError_t e = cudaMemsetAsync(w, 0, L.mask + mask_bytes, stream);
+  const bool gemv = (path == kPathDecode) || (path == kPathAuto && T <= kDecodeMaxT);
+  // the decode prep kernel clears the status word itself and keeps the mask
+  // in shared memory; otherwise status word + mask start at zero
+  const bool small_prep = gemv && T >= 1;
+  cudaError_t e = small_prep ? cudaSuccess : cudaMemsetAsync(w, 0, L.mask + mask_bytes, stream);
   if (e != cudaSuccess) return I8_ERR_CUDA;
   if (T == 0) {
     e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
@@ -170,18 +173,22 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   void* Wo = w + L.Wo;
 
   const uint32_t hb = threshold_bits(threshold, dtype);
-  if (hb == 0xffffffffu)
-    e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
-  else
-    e = launch_outliers(X, dtype, T, K, hb, mask, prefix, idx, n_out, dst, stream);
-  if (e != cudaSuccess || !mark(1)) return I8_ERR_CUDA;
-
-  const bool gemv = (path == kPathDecode) || (path == kPathAuto && T <= kDecodeMaxT);
-  // programmatic launches only directly after one of our kernels
-  const bool after_outliers = (hb != 0xffffffffu);
-  e = launch_rowquant(X, dtype, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, Wf, num_sms,
-                      dst, after_outliers, stream);
-  if (e != cudaSuccess || !mark(2)) return I8_ERR_CUDA;
+  if (small_prep) {
+    // one kernel for the outlier pass and the row quantisation
+    e = launch_prep_small(X, dtype, T, K, hb, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, dst, stream);
+    if (e != cudaSuccess || !mark(1) || !mark(2)) return I8_ERR_CUDA;
+  } else {
+    if (hb == 0xffffffffu)
+      e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
+    else
+      e = launch_outliers(X, dtype, T, K, hb, mask, prefix, idx, n_out, dst, stream);
+    if (e != cudaSuccess || !mark(1)) return I8_ERR_CUDA;
+    // programmatic launches only directly after one of our kernels
+    const bool after_outliers = (hb != 0xffffffffu);
+    e = launch_rowquant(X, dtype, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, Wf,
+                        num_sms, dst, after_outliers, stream);
+    if (e != cudaSuccess || !mark(2)) return I8_ERR_CUDA;
+  }
 
   GemmArgs a;
   a.Xq = Xq;

@@ -63,6 +63,13 @@ __device__ __forceinline__ void store_extra(const YDst& y, int64_t off, TE v) {
     if (d < y.n) static_cast<TE*>(y.p[d])[off] = v;
 }
 
+// Decode prep (1 <= T <= kDecodeMaxT, product by the decode GEMV): outlier
+// mask, idx, n_out and row quantisation in one kernel, one CTA per row; also
+// clears the status word.  hbits == 0xffffffff: no outliers.  No Wo.
+cudaError_t launch_prep_small(const void* X, int dtype, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
+                              uint32_t* prefix, int32_t* idx, int32_t* n_out, int8_t* Xq, float* sA, void* Xo,
+                              int64_t ldo, DevStatus* st, cudaStream_t s);
+
 struct GemmArgs {
   const int8_t* Xq;      // [T,K]
   const int8_t* CB;      // [N,K]

@@ -96,24 +96,17 @@ extern "C" i8_status int8_linear_forward_decode_static(const void* X, int64_t T,
   if (st != I8_OK) return st;
   uint8_t* w = static_cast<uint8_t*>(base);
 
-  // The scratch keeps whatever the previous call left: the status word and the
-  // outlier bitmask must start at zero.
-  if (cudaMemsetAsync(w, 0, L.sA, stream) != cudaSuccess) return I8_ERR_CUDA;
+  // The scratch keeps whatever the previous call left; the prep kernel
+  // rebuilds the outlier bitmask from scratch and clears the status word.
   DevStatus* dst = reinterpret_cast<DevStatus*>(w + L.status);
   uint32_t* mask = reinterpret_cast<uint32_t*>(w + L.mask);
   float* sA = reinterpret_cast<float*>(w + L.sA);
   int8_t* Xq = reinterpret_cast<int8_t*>(w + L.Xq);
   void* Xo = w + L.Xo;
 
-  cudaError_t e;
   const uint32_t hb = int8_outlier_threshold_bits(threshold);
-  if (hb == 0xffffffffu)
-    e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
-  else
-    e = launch_outliers(X, kF16, T, K, hb, mask, mask + (K + 31) / 32, idx, n_out, dst, stream);
-  if (e != cudaSuccess) return I8_ERR_CUDA;
-  e = launch_rowquant(X, kF16, T, K, mask, mask + (K + 31) / 32, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, nullptr,
-                      false, nullptr, num_sms, dst, hb != 0xffffffffu, stream);
+  const cudaError_t e = launch_prep_small(X, kF16, T, K, hb, mask, mask + (K + 31) / 32, idx, n_out, Xq, sA, Xo,
+                                          L.ldo, dst, stream);
   if (e != cudaSuccess) return I8_ERR_CUDA;
 
   GemmArgs a;
@@ -134,6 +127,6 @@ extern "C" i8_status int8_linear_forward_decode_static(const void* X, int64_t T,
   a.N = N;
   a.K = K;
   a.mode = 0;
-  a.pdl = true;  // follows the row quantisation kernel
+  a.pdl = true;  // follows the prep kernel
   return launch_gemv_decode(a, num_sms, stream) == cudaSuccess ? I8_OK : I8_ERR_CUDA;
 }

@@ -276,17 +276,57 @@ __device__ __forceinline__ uint2 row_codes_fast(const uint4& v, uint32_t mb, flo
   return make_uint2(w[0], w[1]);
 }
 
-// Scatter the outlier entries of one 8-column chunk into the Xo row.
-template <typename TE>
+// Scatter the outlier entries of one 8-column chunk into the Xo row.  mask and
+// prefix are in global memory (read-only path) or, with kShared, in shared
+// memory.
+template <typename TE, bool kShared = false>
 __device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, int64_t chunk, const uint32_t* mask,
                                                  const uint32_t* prefix, TE* xo_row) {
   const TE* h = reinterpret_cast<const TE*>(&v);
-  const uint32_t mw = __ldg(&mask[chunk >> 2]);
-  const uint32_t base = __ldg(&prefix[chunk >> 2]);
+  const uint32_t mw = kShared ? mask[chunk >> 2] : __ldg(&mask[chunk >> 2]);
+  const uint32_t base = kShared ? prefix[chunk >> 2] : __ldg(&prefix[chunk >> 2]);
   const int sh = static_cast<int>(chunk & 3) * 8;
   #pragma unroll
   for (int e = 0; e < 8; ++e)
     if ((mb >> e) & 1u) xo_row[base + __popc(mw & ((1u << (sh + e)) - 1u))] = h[e];
+}
+
+// Wo[j, o] for the outlier columns, grid-strided over the N x npad elements by
+// the `wo_blocks` CTAs of NT threads that follow the row CTAs: four
+// independent gathers per thread in flight.
+template <typename TE, int NT>
+__device__ __forceinline__ void wo_gather(int64_t wblk, int64_t wo_blocks, int n_out, int64_t npad,
+                                          const int32_t* __restrict__ idx, const int8_t* __restrict__ CB,
+                                          const float* __restrict__ SCB, int64_t N, int64_t K, TE* __restrict__ Wo,
+                                          int64_t ldo, const TE* __restrict__ Wf) {
+  using E = Elem<TE>;
+  if (n_out == 0) return;
+  const int64_t total = N * npad;
+  const int64_t stride = wo_blocks * NT * kWoUnroll;
+  for (int64_t e0 = wblk * NT * kWoUnroll + threadIdx.x; e0 < total; e0 += stride) {
+    int8_t cbv[kWoUnroll];
+    TE wfv[kWoUnroll];
+    int64_t jj[kWoUnroll], oo[kWoUnroll];
+    #pragma unroll
+    for (int u = 0; u < kWoUnroll; ++u) {
+      const int64_t e = e0 + static_cast<int64_t>(u) * NT;
+      jj[u] = e / npad;
+      oo[u] = e - jj[u] * npad;
+      const bool live = e < total && oo[u] < n_out;
+      cbv[u] = (live && Wf == nullptr) ? __ldg(&CB[jj[u] * K + __ldg(&idx[oo[u]])]) : int8_t(0);
+      wfv[u] = (live && Wf != nullptr) ? Wf[jj[u] * K + __ldg(&idx[oo[u]])] : E::from_float(0.0f);
+    }
+    #pragma unroll
+    for (int u = 0; u < kWoUnroll; ++u) {
+      const int64_t e = e0 + static_cast<int64_t>(u) * NT;
+      if (e < total) {
+        TE v = wfv[u];
+        if (oo[u] < n_out && Wf == nullptr)
+          v = E::from_float(__fdiv_rn(__fmul_rn(static_cast<float>(cbv[u]), __ldg(&SCB[jj[u]])), 127.0f));
+        Wo[jj[u] * ldo + oo[u]] = v;
+      }
+    }
+  }
 }
 
 template <typename TE>
@@ -304,35 +344,8 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
   const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
 
   if (static_cast<int64_t>(blockIdx.x) >= row_blocks) {
-    // ---- Wo rows ----
-    if (n_out == 0) return;
-    const int64_t total = N * npad;
-    const int64_t stride = wo_blocks * kRowThreads * kWoUnroll;
-    for (int64_t e0 = (static_cast<int64_t>(blockIdx.x) - row_blocks) * kRowThreads * kWoUnroll + threadIdx.x;
-         e0 < total; e0 += stride) {
-      int8_t cbv[kWoUnroll];
-      TE wfv[kWoUnroll];
-      int64_t jj[kWoUnroll], oo[kWoUnroll];
-      #pragma unroll
-      for (int u = 0; u < kWoUnroll; ++u) {
-        const int64_t e = e0 + static_cast<int64_t>(u) * kRowThreads;
-        jj[u] = e / npad;
-        oo[u] = e - jj[u] * npad;
-        const bool live = e < total && oo[u] < n_out;
-        cbv[u] = (live && Wf == nullptr) ? __ldg(&CB[jj[u] * K + __ldg(&idx[oo[u]])]) : int8_t(0);
-        wfv[u] = (live && Wf != nullptr) ? Wf[jj[u] * K + __ldg(&idx[oo[u]])] : E::from_float(0.0f);
-      }
-      #pragma unroll
-      for (int u = 0; u < kWoUnroll; ++u) {
-        const int64_t e = e0 + static_cast<int64_t>(u) * kRowThreads;
-        if (e < total) {
-          TE v = wfv[u];
-          if (oo[u] < n_out && Wf == nullptr)
-            v = E::from_float(__fdiv_rn(__fmul_rn(static_cast<float>(cbv[u]), __ldg(&SCB[jj[u]])), 127.0f));
-          Wo[jj[u] * ldo + oo[u]] = v;
-        }
-      }
-    }
+    wo_gather<TE, kRowThreads>(static_cast<int64_t>(blockIdx.x) - row_blocks, wo_blocks, n_out, npad, idx, CB, SCB,
+                               N, K, Wo, ldo, Wf);
     return;
   }
 
@@ -383,15 +396,241 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
   for (int64_t o = n_out + lane; o < npad; o += 32) xo_row[o] = E::from_float(0.0f);
 }
 
+// Few rows (fewer warp-per-row CTAs than SMs): one 512-thread CTA per row, so
+// that a pass over the row needs about one round of loads instead of K/2048
+// rounds by a single warp; the absmax is reduced across the CTA.
+constexpr int kRowCtaThreads = 512;
+constexpr int kRowCtaUnroll = 4;
+
 template <typename TE>
-static cudaError_t launch_rowquant_t(const cudaLaunchConfig_t& cfg, const void* X, int64_t T, int64_t K,
-                                     const uint32_t* mask, const uint32_t* prefix, const int32_t* idx,
+__global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
+    const TE* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
+    const uint32_t* __restrict__ prefix, const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p,
+    int8_t* __restrict__ Xq, float* __restrict__ sA, TE* __restrict__ Xo, int64_t ldo,
+    const int8_t* __restrict__ CB, const float* __restrict__ SCB, int64_t N, TE* __restrict__ Wo,
+    const TE* __restrict__ Wf, int64_t row_blocks, int64_t wo_blocks) {
+  using E = Elem<TE>;
+  __shared__ uint32_t s_max[kRowCtaThreads / 32];
+  griddep_launch_dependents();
+  griddep_wait();  // mask, prefix, idx, n_out come from the outlier pass
+  const int n_out = *n_out_p;
+  const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
+  if (static_cast<int64_t>(blockIdx.x) >= row_blocks) {
+    wo_gather<TE, kRowCtaThreads>(static_cast<int64_t>(blockIdx.x) - row_blocks, wo_blocks, n_out, npad, idx, CB,
+                                  SCB, N, K, Wo, ldo, Wf);
+    return;
+  }
+  const int64_t t = blockIdx.x;
+  const int64_t nv = K / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(X + t * K);
+  constexpr int64_t kStep = static_cast<int64_t>(kRowCtaThreads) * kRowCtaUnroll;
+  uint32_t mmax = 0;
+  for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
+    uint4 v[kRowCtaUnroll];
+    #pragma unroll
+    for (int u = 0; u < kRowCtaUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+    #pragma unroll
+    for (int u = 0; u < kRowCtaUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+      if (c < nv) mmax = max(mmax, chunk_max_mag_kept<TE>(v[u], mask_byte(mask, c)));
+    }
+  }
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = mmax;
+  __syncthreads();
+  mmax = 0;
+  #pragma unroll
+  for (int w = 0; w < kRowCtaThreads / 32; ++w) mmax = max(mmax, s_max[w]);
+  const float absmax = E::mag_to_float(mmax);
+  const float inv = scale_inv(absmax);
+  if (threadIdx.x == 0) sA[t] = absmax;
+
+  uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
+  TE* xo_row = Xo + t * ldo;
+  for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
+    uint4 v[kRowCtaUnroll];
+    #pragma unroll
+    for (int u = 0; u < kRowCtaUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+    #pragma unroll
+    for (int u = 0; u < kRowCtaUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+      if (c < nv) {
+        const uint32_t mb = mask_byte(mask, c);
+        dst[c] = row_codes_fast<TE>(v[u], mb, inv);
+        if (mb) scatter_outliers<TE>(v[u], mb, c, mask, prefix, xo_row);
+      }
+    }
+  }
+  for (int64_t o = n_out + threadIdx.x; o < npad; o += kRowCtaThreads) xo_row[o] = E::from_float(0.0f);
+}
+
+// ---------------------------------------------------------------------------
+// Decode prep (T <= 16, weight-streaming product): the outlier pass and the
+// row quantisation in one kernel, one 512-thread CTA per token row.  Every
+// CTA rebuilds the column mask from all T rows (at most 16 x K x 2 bytes, read
+// through L2) into shared memory, with the per-word prefix counts, and then
+// quantises its row.  CTA 0 also publishes mask, prefix, idx and n_out and
+// clears the status word, so the forward needs no memset and no separate
+// outlier launch.  hbits == 0xffffffff means "no outliers".
+// ---------------------------------------------------------------------------
+constexpr int kSmallMaxK = 131072;
+
+template <typename TE>
+__global__ void __launch_bounds__(kRowCtaThreads) prep_small_kernel(
+    const TE* __restrict__ X, int64_t T, int64_t K, uint32_t hbits, uint32_t* __restrict__ mask,
+    uint32_t* __restrict__ prefix, int32_t* __restrict__ idx, int32_t* __restrict__ n_out_p, int8_t* __restrict__ Xq,
+    float* __restrict__ sA, TE* __restrict__ Xo, int64_t ldo, DevStatus* st) {
+  using E = Elem<TE>;
+  __shared__ uint32_t s_mask[kSmallMaxK / 32];
+  __shared__ uint32_t s_prefix[kSmallMaxK / 32];
+  __shared__ int s_scan[kRowCtaThreads];
+  __shared__ uint32_t s_max[kRowCtaThreads / 32];
+  griddep_launch_dependents();  // the product kernel may start its prologue
+  const int64_t nv = K / 8;
+  const int64_t nw = (K + 31) / 32;
+  const bool on = hbits != 0xffffffffu;
+  const uint32_t h2 = hbits | (hbits << 16);
+  for (int64_t w = threadIdx.x; w < nw; w += kRowCtaThreads) s_mask[w] = 0;
+  __syncthreads();
+  // mask: column chunk c is flagged from all T rows
+  if (on) {
+    for (int64_t c = threadIdx.x; c < nv; c += kRowCtaThreads) {
+      uint32_t bits = 0;
+      int64_t r = 0;
+      for (; r + 4 <= T; r += 4) {
+        uint4 v[4];
+        #pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(X + (r + u) * K) + c);
+        #pragma unroll
+        for (int u = 0; u < 4; ++u) bits |= flag_bits8<TE>(v[u], h2);
+      }
+      for (; r < T; ++r) bits |= flag_bits8<TE>(__ldg(reinterpret_cast<const uint4*>(X + r * K) + c), h2);
+      if (bits) atomicOr(&s_mask[c >> 2], bits << ((c & 3) * 8));
+    }
+  }
+  __syncthreads();
+  // prefix counts: thread i owns a contiguous run of mask words
+  const int64_t per = (nw + kRowCtaThreads - 1) / kRowCtaThreads;
+  const int64_t w0 = threadIdx.x * per;
+  const int64_t w1 = min(nw, w0 + per);
+  int cnt = 0;
+  for (int64_t w = w0; w < w1; ++w) cnt += __popc(s_mask[w]);
+  s_scan[threadIdx.x] = cnt;
+  __syncthreads();
+  for (int off = 1; off < kRowCtaThreads; off <<= 1) {
+    const int v = (static_cast<int>(threadIdx.x) >= off) ? s_scan[threadIdx.x - off] : 0;
+    __syncthreads();
+    s_scan[threadIdx.x] += v;
+    __syncthreads();
+  }
+  const int n_out = s_scan[kRowCtaThreads - 1];
+  int pos = s_scan[threadIdx.x] - cnt;
+  for (int64_t w = w0; w < w1; ++w) {
+    s_prefix[w] = static_cast<uint32_t>(pos);
+    if (blockIdx.x == 0) {
+      uint32_t m = s_mask[w];
+      mask[w] = m;
+      prefix[w] = static_cast<uint32_t>(pos);
+      while (m) {
+        const int b = __ffs(m) - 1;
+        m &= m - 1;
+        idx[pos++] = static_cast<int32_t>(w * 32 + b);
+      }
+    } else {
+      pos += __popc(s_mask[w]);
+    }
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *n_out_p = n_out;
+    st->error = 0;
+    st->where = 0;
+  }
+  __syncthreads();
+
+  // this CTA's row, as rowquant_cta_kernel with the mask from shared memory
+  const int64_t t = blockIdx.x;
+  const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
+  const uint4* src = reinterpret_cast<const uint4*>(X + t * K);
+  const uint8_t* mb8 = reinterpret_cast<const uint8_t*>(s_mask);
+  constexpr int64_t kStep = static_cast<int64_t>(kRowCtaThreads) * kRowCtaUnroll;
+  uint32_t mmax = 0;
+  for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
+    uint4 v[kRowCtaUnroll];
+    #pragma unroll
+    for (int u = 0; u < kRowCtaUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+    #pragma unroll
+    for (int u = 0; u < kRowCtaUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+      if (c < nv) mmax = max(mmax, chunk_max_mag_kept<TE>(v[u], mb8[c]));
+    }
+  }
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = mmax;
+  __syncthreads();
+  mmax = 0;
+  #pragma unroll
+  for (int w = 0; w < kRowCtaThreads / 32; ++w) mmax = max(mmax, s_max[w]);
+  const float absmax = E::mag_to_float(mmax);
+  const float inv = scale_inv(absmax);
+  if (threadIdx.x == 0) sA[t] = absmax;
+  uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
+  TE* xo_row = Xo + t * ldo;
+  for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
+    uint4 v[kRowCtaUnroll];
+    #pragma unroll
+    for (int u = 0; u < kRowCtaUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+    #pragma unroll
+    for (int u = 0; u < kRowCtaUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+      if (c < nv) {
+        const uint32_t mb = mb8[c];
+        dst[c] = row_codes_fast<TE>(v[u], mb, inv);
+        if (mb) scatter_outliers<TE, true>(v[u], mb, c, s_mask, s_prefix, xo_row);
+      }
+    }
+  }
+  for (int64_t o = n_out + threadIdx.x; o < npad; o += kRowCtaThreads) xo_row[o] = E::from_float(0.0f);
+}
+
+cudaError_t launch_prep_small(const void* X, int dtype, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
+                              uint32_t* prefix, int32_t* idx, int32_t* n_out, int8_t* Xq, float* sA, void* Xo,
+                              int64_t ldo, DevStatus* st, cudaStream_t s) {
+  if (T < 1 || T > kDecodeMaxT || K > kSmallMaxK) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(T));
+  if (dtype == kBF16)
+    prep_small_kernel<__nv_bfloat16><<<grid, kRowCtaThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(X), T, K, hbits, mask, prefix, idx, n_out, Xq, sA,
+        static_cast<__nv_bfloat16*>(Xo), ldo, st);
+  else
+    prep_small_kernel<__half><<<grid, kRowCtaThreads, 0, s>>>(static_cast<const __half*>(X), T, K, hbits, mask,
+                                                              prefix, idx, n_out, Xq, sA, static_cast<__half*>(Xo),
+                                                              ldo, st);
+  return cudaGetLastError();
+}
+
+template <typename TE>
+static cudaError_t launch_rowquant_t(const cudaLaunchConfig_t& cfg, bool cta_rows, const void* X, int64_t T,
+                                     int64_t K, const uint32_t* mask, const uint32_t* prefix, const int32_t* idx,
                                      const int32_t* n_out, int8_t* Xq, float* sA, void* Xo, int64_t ldo,
                                      const int8_t* CB, const float* SCB, int64_t N, void* Wo, const void* Wf,
                                      int64_t row_blocks, int64_t wo_blocks) {
-  return cudaLaunchKernelEx(&cfg, rowquant_kernel<TE>, static_cast<const TE*>(X), T, K, mask, prefix, idx, n_out, Xq,
-                            sA, static_cast<TE*>(Xo), ldo, CB, SCB, N, static_cast<TE*>(Wo),
-                            static_cast<const TE*>(Wf), row_blocks, wo_blocks);
+  return cudaLaunchKernelEx(&cfg, cta_rows ? rowquant_cta_kernel<TE> : rowquant_kernel<TE>,
+                            static_cast<const TE*>(X), T, K, mask, prefix, idx, n_out, Xq, sA, static_cast<TE*>(Xo),
+                            ldo, CB, SCB, N, static_cast<TE*>(Wo), static_cast<const TE*>(Wf), row_blocks, wo_blocks);
 }
 
 cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, const uint32_t* mask,
@@ -399,14 +638,17 @@ cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, cons
                             void* Xo, int64_t ldo, const int8_t* CB, const float* SCB, int64_t N, void* Wo,
                             bool with_wo, const void* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s) {
   (void)st;
+  // Warp-per-row CTAs while they fill the SMs; one CTA per row below that.
+  const bool cta_rows = (T + kRowWarps - 1) / kRowWarps < num_sms;
+  const int threads = cta_rows ? kRowCtaThreads : kRowThreads;
   int64_t wo_blocks = 0;
   if (with_wo) {
-    wo_blocks = (N * 64 + kRowThreads * kWoUnroll - 1) / (kRowThreads * kWoUnroll);
-    const int64_t cap = static_cast<int64_t>(num_sms) * 4;
+    wo_blocks = (N * 64 + threads * kWoUnroll - 1) / (threads * kWoUnroll);
+    const int64_t cap = static_cast<int64_t>(num_sms) * (cta_rows ? 2 : 4);
     if (wo_blocks > cap) wo_blocks = cap;
     if (wo_blocks < 1) wo_blocks = 1;
   }
-  const int64_t row_blocks = (T + kRowWarps - 1) / kRowWarps;
+  const int64_t row_blocks = cta_rows ? T : (T + kRowWarps - 1) / kRowWarps;
   const int64_t blocks = row_blocks + wo_blocks;
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
@@ -415,15 +657,15 @@ cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
-  cfg.blockDim = dim3(kRowThreads, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   if (dtype == kBF16)
-    return launch_rowquant_t<__nv_bfloat16>(cfg, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N, Wo,
-                                            Wf, row_blocks, wo_blocks);
-  return launch_rowquant_t<__half>(cfg, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N, Wo, Wf,
-                                   row_blocks, wo_blocks);
+    return launch_rowquant_t<__nv_bfloat16>(cfg, cta_rows, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB,
+                                            SCB, N, Wo, Wf, row_blocks, wo_blocks);
+  return launch_rowquant_t<__half>(cfg, cta_rows, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N,
+                                   Wo, Wf, row_blocks, wo_blocks);
 }
 
 }  // namespace i8mp
