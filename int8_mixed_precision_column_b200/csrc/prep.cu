@@ -226,14 +226,13 @@ cudaError_t launch_outliers(const void* X, int dtype, int64_t T, int64_t K, uint
 //           registers, rank = prefix[word] + popc(lower bits of the word).
 // Xo is zero-padded to the next multiple of 64 (the 16-bit outlier K-block).
 // Wo blocks (blockIdx >= row blocks): Wo[j, o] = TE((CB[j, idx[o]] * SCB[j]) / 127)
-// with the same padding, four independent gathers per thread in flight (only
-// when the tensor-core product consumes Wo).  With a 16-bit weight Wf (the
+// with the same padding, 8 outputs per lane and 16-byte stores (only when the
+// tensor-core product consumes Wo).  With a 16-bit weight Wf (the
 // has_fp16_weights=True layer) Wo[j, o] = Wf[j, idx[o]] instead.
 // ---------------------------------------------------------------------------
 constexpr int kRowThreads = 256;
 constexpr int kRowWarps = kRowThreads / 32;
 constexpr int kRowUnroll = 8;
-constexpr int kWoUnroll = 4;
 
 __device__ __forceinline__ uint32_t mask_byte(const uint32_t* mask, int64_t chunk) {
   return (__ldg(&mask[chunk >> 2]) >> ((chunk & 3) * 8)) & 0xffu;
@@ -291,9 +290,11 @@ __device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, in
     if ((mb >> e) & 1u) xo_row[base + __popc(mw & ((1u << (sh + e)) - 1u))] = h[e];
 }
 
-// Wo[j, o] for the outlier columns, grid-strided over the N x npad elements by
-// the `wo_blocks` CTAs of NT threads that follow the row CTAs: four
-// independent gathers per thread in flight.
+// Wo[j, o] for the outlier columns, by the `wo_blocks` CTAs of NT threads
+// that follow the row CTAs.  A warp covers whole rows j: its lanes split into
+// groups of L = min(32, npad/8 rounded up to a power of two) lanes per row,
+// each lane builds 8 consecutive outputs and writes them with one 16-byte
+// store (npad is a multiple of 64, ldo of 64: rows stay 16-byte aligned).
 template <typename TE, int NT>
 __device__ __forceinline__ void wo_gather(int64_t wblk, int64_t wo_blocks, int n_out, int64_t npad,
                                           const int32_t* __restrict__ idx, const int8_t* __restrict__ CB,
@@ -301,30 +302,40 @@ __device__ __forceinline__ void wo_gather(int64_t wblk, int64_t wo_blocks, int n
                                           int64_t ldo, const TE* __restrict__ Wf) {
   using E = Elem<TE>;
   if (n_out == 0) return;
-  const int64_t total = N * npad;
-  const int64_t stride = wo_blocks * NT * kWoUnroll;
-  for (int64_t e0 = wblk * NT * kWoUnroll + threadIdx.x; e0 < total; e0 += stride) {
-    int8_t cbv[kWoUnroll];
-    TE wfv[kWoUnroll];
-    int64_t jj[kWoUnroll], oo[kWoUnroll];
-    #pragma unroll
-    for (int u = 0; u < kWoUnroll; ++u) {
-      const int64_t e = e0 + static_cast<int64_t>(u) * NT;
-      jj[u] = e / npad;
-      oo[u] = e - jj[u] * npad;
-      const bool live = e < total && oo[u] < n_out;
-      cbv[u] = (live && Wf == nullptr) ? __ldg(&CB[jj[u] * K + __ldg(&idx[oo[u]])]) : int8_t(0);
-      wfv[u] = (live && Wf != nullptr) ? Wf[jj[u] * K + __ldg(&idx[oo[u]])] : E::from_float(0.0f);
-    }
-    #pragma unroll
-    for (int u = 0; u < kWoUnroll; ++u) {
-      const int64_t e = e0 + static_cast<int64_t>(u) * NT;
-      if (e < total) {
-        TE v = wfv[u];
-        if (oo[u] < n_out && Wf == nullptr)
-          v = E::from_float(__fdiv_rn(__fmul_rn(static_cast<float>(cbv[u]), __ldg(&SCB[jj[u]])), 127.0f));
-        Wo[jj[u] * ldo + oo[u]] = v;
+  const int lane = threadIdx.x & 31;
+  const int chunks = static_cast<int>(npad / 8);
+  int lpr_log = 0;  // log2 of lanes per row
+  while ((1 << lpr_log) < chunks && lpr_log < 5) ++lpr_log;
+  const int lpr = 1 << lpr_log;
+  const int sub = lane >> lpr_log;   // row within the warp's group
+  const int l = lane & (lpr - 1);
+  const int64_t rows_per_warp = 32 >> lpr_log;
+  const int64_t warps = wo_blocks * (NT / 32);
+  const int64_t warp = wblk * (NT / 32) + (threadIdx.x >> 5);
+  for (int64_t j = warp * rows_per_warp + sub; j < N; j += warps * rows_per_warp) {
+    const float scb = Wf == nullptr ? __ldg(&SCB[j]) : 0.0f;
+    const int8_t* cbrow = CB + j * K;
+    const TE* wfrow = Wf == nullptr ? nullptr : Wf + j * K;
+    TE* worow = Wo + j * ldo;
+    for (int c = l; c < chunks; c += lpr) {
+      const int o0 = c * 8;
+      uint32_t packed[4];
+      #pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        float f[2];
+        #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int o = o0 + i + h;
+          f[h] = 0.0f;
+          if (o < n_out) {
+            const int col = __ldg(&idx[o]);
+            f[h] = wfrow != nullptr ? E::to_float(wfrow[col])
+                                    : __fdiv_rn(__fmul_rn(static_cast<float>(__ldg(&cbrow[col])), scb), 127.0f);
+          }
+        }
+        packed[i >> 1] = E::pack2(f[0], f[1]);
       }
+      *reinterpret_cast<uint4*>(worow + o0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
   }
 }
@@ -396,13 +407,16 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
   for (int64_t o = n_out + lane; o < npad; o += 32) xo_row[o] = E::from_float(0.0f);
 }
 
-// Few rows (fewer warp-per-row CTAs than SMs): one 512-thread CTA per row, so
-// that a pass over the row needs about one round of loads instead of K/2048
-// rounds by a single warp; the absmax is reduced across the CTA.
-constexpr int kRowCtaThreads = 512;
-constexpr int kRowCtaUnroll = 4;
+// One 256-thread CTA per row: a pass over the row needs about one round of
+// loads, and the absmax is reduced across the CTA.  kResident (rows of at
+// most 256 x 8 chunks, K <= 16384): the row is loaded once and stays in
+// registers between the absmax and the codes, so X is read once.  (Measured
+// against 512 x 4 and 128 x 16: equal at K = 14336, 15 % faster at K = 4096.)
+constexpr int kRowCtaThreads = 256;
+constexpr int kRowCtaUnroll = 8;
+constexpr int64_t kResidentMaxK = static_cast<int64_t>(kRowCtaThreads) * kRowCtaUnroll * 8;
 
-template <typename TE>
+template <typename TE, bool kResident>
 __global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
     const TE* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
     const uint32_t* __restrict__ prefix, const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p,
@@ -425,18 +439,21 @@ __global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
   const uint4* src = reinterpret_cast<const uint4*>(X + t * K);
   constexpr int64_t kStep = static_cast<int64_t>(kRowCtaThreads) * kRowCtaUnroll;
   uint32_t mmax = 0;
+  uint4 v[kRowCtaUnroll];   // with kResident: the whole row share of this thread
+  uint32_t mbs[kRowCtaUnroll];
   for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
-    uint4 v[kRowCtaUnroll];
     #pragma unroll
     for (int u = 0; u < kRowCtaUnroll; ++u) {
       const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
       v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+      mbs[u] = (c < nv) ? mask_byte(mask, c) : 0u;
     }
     #pragma unroll
     for (int u = 0; u < kRowCtaUnroll; ++u) {
       const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
-      if (c < nv) mmax = max(mmax, chunk_max_mag_kept<TE>(v[u], mask_byte(mask, c)));
+      if (c < nv) mmax = max(mmax, chunk_max_mag_kept<TE>(v[u], mbs[u]));
     }
+    if constexpr (kResident) break;
   }
   #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
@@ -452,21 +469,23 @@ __global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
   uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
   TE* xo_row = Xo + t * ldo;
   for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
-    uint4 v[kRowCtaUnroll];
-    #pragma unroll
-    for (int u = 0; u < kRowCtaUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
-      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    if constexpr (!kResident) {
+      #pragma unroll
+      for (int u = 0; u < kRowCtaUnroll; ++u) {
+        const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+        v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+        mbs[u] = (c < nv) ? mask_byte(mask, c) : 0u;
+      }
     }
     #pragma unroll
     for (int u = 0; u < kRowCtaUnroll; ++u) {
       const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
       if (c < nv) {
-        const uint32_t mb = mask_byte(mask, c);
-        dst[c] = row_codes_fast<TE>(v[u], mb, inv);
-        if (mb) scatter_outliers<TE>(v[u], mb, c, mask, prefix, xo_row);
+        dst[c] = row_codes_fast<TE>(v[u], mbs[u], inv);
+        if (mbs[u]) scatter_outliers<TE>(v[u], mbs[u], c, mask, prefix, xo_row);
       }
     }
+    if constexpr (kResident) break;
   }
   for (int64_t o = n_out + threadIdx.x; o < npad; o += kRowCtaThreads) xo_row[o] = E::from_float(0.0f);
 }
@@ -481,27 +500,29 @@ __global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
 // outlier launch.  hbits == 0xffffffff means "no outliers".
 // ---------------------------------------------------------------------------
 constexpr int kSmallMaxK = 131072;
+constexpr int kSmallThreads = 512;
+constexpr int kSmallUnroll = 4;
 
 template <typename TE>
-__global__ void __launch_bounds__(kRowCtaThreads) prep_small_kernel(
+__global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
     const TE* __restrict__ X, int64_t T, int64_t K, uint32_t hbits, uint32_t* __restrict__ mask,
     uint32_t* __restrict__ prefix, int32_t* __restrict__ idx, int32_t* __restrict__ n_out_p, int8_t* __restrict__ Xq,
     float* __restrict__ sA, TE* __restrict__ Xo, int64_t ldo, DevStatus* st) {
   using E = Elem<TE>;
   __shared__ uint32_t s_mask[kSmallMaxK / 32];
   __shared__ uint32_t s_prefix[kSmallMaxK / 32];
-  __shared__ int s_scan[kRowCtaThreads];
-  __shared__ uint32_t s_max[kRowCtaThreads / 32];
+  __shared__ int s_scan[kSmallThreads];
+  __shared__ uint32_t s_max[kSmallThreads / 32];
   griddep_launch_dependents();  // the product kernel may start its prologue
   const int64_t nv = K / 8;
   const int64_t nw = (K + 31) / 32;
   const bool on = hbits != 0xffffffffu;
   const uint32_t h2 = hbits | (hbits << 16);
-  for (int64_t w = threadIdx.x; w < nw; w += kRowCtaThreads) s_mask[w] = 0;
+  for (int64_t w = threadIdx.x; w < nw; w += kSmallThreads) s_mask[w] = 0;
   __syncthreads();
   // mask: column chunk c is flagged from all T rows
   if (on) {
-    for (int64_t c = threadIdx.x; c < nv; c += kRowCtaThreads) {
+    for (int64_t c = threadIdx.x; c < nv; c += kSmallThreads) {
       uint32_t bits = 0;
       int64_t r = 0;
       for (; r + 4 <= T; r += 4) {
@@ -517,20 +538,20 @@ __global__ void __launch_bounds__(kRowCtaThreads) prep_small_kernel(
   }
   __syncthreads();
   // prefix counts: thread i owns a contiguous run of mask words
-  const int64_t per = (nw + kRowCtaThreads - 1) / kRowCtaThreads;
+  const int64_t per = (nw + kSmallThreads - 1) / kSmallThreads;
   const int64_t w0 = threadIdx.x * per;
   const int64_t w1 = min(nw, w0 + per);
   int cnt = 0;
   for (int64_t w = w0; w < w1; ++w) cnt += __popc(s_mask[w]);
   s_scan[threadIdx.x] = cnt;
   __syncthreads();
-  for (int off = 1; off < kRowCtaThreads; off <<= 1) {
+  for (int off = 1; off < kSmallThreads; off <<= 1) {
     const int v = (static_cast<int>(threadIdx.x) >= off) ? s_scan[threadIdx.x - off] : 0;
     __syncthreads();
     s_scan[threadIdx.x] += v;
     __syncthreads();
   }
-  const int n_out = s_scan[kRowCtaThreads - 1];
+  const int n_out = s_scan[kSmallThreads - 1];
   int pos = s_scan[threadIdx.x] - cnt;
   for (int64_t w = w0; w < w1; ++w) {
     s_prefix[w] = static_cast<uint32_t>(pos);
@@ -559,18 +580,18 @@ __global__ void __launch_bounds__(kRowCtaThreads) prep_small_kernel(
   const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
   const uint4* src = reinterpret_cast<const uint4*>(X + t * K);
   const uint8_t* mb8 = reinterpret_cast<const uint8_t*>(s_mask);
-  constexpr int64_t kStep = static_cast<int64_t>(kRowCtaThreads) * kRowCtaUnroll;
+  constexpr int64_t kStep = static_cast<int64_t>(kSmallThreads) * kSmallUnroll;
   uint32_t mmax = 0;
   for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
-    uint4 v[kRowCtaUnroll];
+    uint4 v[kSmallUnroll];
     #pragma unroll
-    for (int u = 0; u < kRowCtaUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+    for (int u = 0; u < kSmallUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kSmallThreads) * u;
       v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
     }
     #pragma unroll
-    for (int u = 0; u < kRowCtaUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+    for (int u = 0; u < kSmallUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kSmallThreads) * u;
       if (c < nv) mmax = max(mmax, chunk_max_mag_kept<TE>(v[u], mb8[c]));
     }
   }
@@ -580,22 +601,22 @@ __global__ void __launch_bounds__(kRowCtaThreads) prep_small_kernel(
   __syncthreads();
   mmax = 0;
   #pragma unroll
-  for (int w = 0; w < kRowCtaThreads / 32; ++w) mmax = max(mmax, s_max[w]);
+  for (int w = 0; w < kSmallThreads / 32; ++w) mmax = max(mmax, s_max[w]);
   const float absmax = E::mag_to_float(mmax);
   const float inv = scale_inv(absmax);
   if (threadIdx.x == 0) sA[t] = absmax;
   uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
   TE* xo_row = Xo + t * ldo;
   for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
-    uint4 v[kRowCtaUnroll];
+    uint4 v[kSmallUnroll];
     #pragma unroll
-    for (int u = 0; u < kRowCtaUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+    for (int u = 0; u < kSmallUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kSmallThreads) * u;
       v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
     }
     #pragma unroll
-    for (int u = 0; u < kRowCtaUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+    for (int u = 0; u < kSmallUnroll; ++u) {
+      const int64_t c = c0 + static_cast<int64_t>(kSmallThreads) * u;
       if (c < nv) {
         const uint32_t mb = mb8[c];
         dst[c] = row_codes_fast<TE>(v[u], mb, inv);
@@ -603,7 +624,7 @@ __global__ void __launch_bounds__(kRowCtaThreads) prep_small_kernel(
       }
     }
   }
-  for (int64_t o = n_out + threadIdx.x; o < npad; o += kRowCtaThreads) xo_row[o] = E::from_float(0.0f);
+  for (int64_t o = n_out + threadIdx.x; o < npad; o += kSmallThreads) xo_row[o] = E::from_float(0.0f);
 }
 
 cudaError_t launch_prep_small(const void* X, int dtype, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
@@ -612,23 +633,26 @@ cudaError_t launch_prep_small(const void* X, int dtype, int64_t T, int64_t K, ui
   if (T < 1 || T > kDecodeMaxT || K > kSmallMaxK) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(T));
   if (dtype == kBF16)
-    prep_small_kernel<__nv_bfloat16><<<grid, kRowCtaThreads, 0, s>>>(
+    prep_small_kernel<__nv_bfloat16><<<grid, kSmallThreads, 0, s>>>(
         static_cast<const __nv_bfloat16*>(X), T, K, hbits, mask, prefix, idx, n_out, Xq, sA,
         static_cast<__nv_bfloat16*>(Xo), ldo, st);
   else
-    prep_small_kernel<__half><<<grid, kRowCtaThreads, 0, s>>>(static_cast<const __half*>(X), T, K, hbits, mask,
+    prep_small_kernel<__half><<<grid, kSmallThreads, 0, s>>>(static_cast<const __half*>(X), T, K, hbits, mask,
                                                               prefix, idx, n_out, Xq, sA, static_cast<__half*>(Xo),
                                                               ldo, st);
   return cudaGetLastError();
 }
 
 template <typename TE>
-static cudaError_t launch_rowquant_t(const cudaLaunchConfig_t& cfg, bool cta_rows, const void* X, int64_t T,
+static cudaError_t launch_rowquant_t(const cudaLaunchConfig_t& cfg, bool cta_rows, bool resident, const void* X,
+                                     int64_t T,
                                      int64_t K, const uint32_t* mask, const uint32_t* prefix, const int32_t* idx,
                                      const int32_t* n_out, int8_t* Xq, float* sA, void* Xo, int64_t ldo,
                                      const int8_t* CB, const float* SCB, int64_t N, void* Wo, const void* Wf,
                                      int64_t row_blocks, int64_t wo_blocks) {
-  return cudaLaunchKernelEx(&cfg, cta_rows ? rowquant_cta_kernel<TE> : rowquant_kernel<TE>,
+  return cudaLaunchKernelEx(&cfg,
+                            cta_rows ? (resident ? rowquant_cta_kernel<TE, true> : rowquant_cta_kernel<TE, false>)
+                                     : rowquant_kernel<TE>,
                             static_cast<const TE*>(X), T, K, mask, prefix, idx, n_out, Xq, sA, static_cast<TE*>(Xo),
                             ldo, CB, SCB, N, static_cast<TE*>(Wo), static_cast<const TE*>(Wf), row_blocks, wo_blocks);
 }
@@ -638,13 +662,16 @@ cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, cons
                             void* Xo, int64_t ldo, const int8_t* CB, const float* SCB, int64_t N, void* Wo,
                             bool with_wo, const void* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s) {
   (void)st;
-  // Warp-per-row CTAs while they fill the SMs; one CTA per row below that.
-  const bool cta_rows = (T + kRowWarps - 1) / kRowWarps < num_sms;
+  // One CTA per row with the row held in registers whenever it fits (X read
+  // once); otherwise warp-per-row CTAs while they fill the SMs, and one CTA
+  // per row (two passes) below that.
+  const bool resident = K <= kResidentMaxK;
+  const bool cta_rows = resident || (T + kRowWarps - 1) / kRowWarps < num_sms;
   const int threads = cta_rows ? kRowCtaThreads : kRowThreads;
   int64_t wo_blocks = 0;
   if (with_wo) {
-    wo_blocks = (N * 64 + threads * kWoUnroll - 1) / (threads * kWoUnroll);
-    const int64_t cap = static_cast<int64_t>(num_sms) * (cta_rows ? 2 : 4);
+    wo_blocks = (N + threads / 32 - 1) / (threads / 32);  // at most one row per warp
+    const int64_t cap = static_cast<int64_t>(num_sms) * 4;
     if (wo_blocks > cap) wo_blocks = cap;
     if (wo_blocks < 1) wo_blocks = 1;
   }
@@ -662,9 +689,9 @@ cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, cons
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   if (dtype == kBF16)
-    return launch_rowquant_t<__nv_bfloat16>(cfg, cta_rows, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB,
+    return launch_rowquant_t<__nv_bfloat16>(cfg, cta_rows, resident, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB,
                                             SCB, N, Wo, Wf, row_blocks, wo_blocks);
-  return launch_rowquant_t<__half>(cfg, cta_rows, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N,
+  return launch_rowquant_t<__half>(cfg, cta_rows, resident, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N,
                                    Wo, Wf, row_blocks, wo_blocks);
 }
 
