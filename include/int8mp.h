@@ -58,6 +58,9 @@ typedef enum i8_status {
   I8_ERR_UNSUPPORTED = 5  /* no sm_100 device, or the driver lacks TMA map encoding */
 } i8_status;
 
+/* 16-bit element types of the *_ex calls (see "16-bit element type" below). */
+enum { I8_DTYPE_F16 = 0, I8_DTYPE_BF16 = 1 };
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* int8_status_string(int status);
 
@@ -199,8 +202,9 @@ i8_status int8_linear_forward_timed(const void* X, int64_t T, int64_t K, const i
  * store CB, SCB and (optionally) the bias in one byte image and read them
  * back, so a layer is loaded without its fp16 weight and without quantising
  * again.  Image (little-endian): "I8MPLYR1", int64 N, int64 K, uint32 flags
- * (bit 0 = bias present), uint32 0, then fp32 SCB[N], fp16 bias[N] if
- * present, int8 CB[N*K] row-major.  Shapes follow the forward's rules.
+ * (bit 0 = bias present, bit 1 = the bias is bf16 rather than fp16), uint32 0,
+ * then fp32 SCB[N], the 16-bit bias[N] if present, int8 CB[N*K] row-major.
+ * Shapes follow the forward's rules.
  * ------------------------------------------------------------------------- */
 
 /* Image size in bytes (0 for an unsupported shape). */
@@ -215,6 +219,14 @@ i8_status int8_layer_unpack_header(const void* buf, size_t bytes, int64_t* N, in
 /* Copies an image's SCB, bias (when present and `bias` is not NULL) and CB
  * into host buffers sized from int8_layer_unpack_header. */
 i8_status int8_layer_unpack(const void* buf, size_t bytes, int8_t* CB, float* SCB, void* bias);
+/* int8_layer_pack with the bias's element type (I8_DTYPE_F16 or I8_DTYPE_BF16,
+ * ignored without a bias) recorded in the image. */
+i8_status int8_layer_pack_ex(const int8_t* CB, const float* SCB, const void* bias, int bias_dtype, int64_t N,
+                             int64_t K, void* out, size_t out_bytes);
+/* int8_layer_unpack_header that also reads the bias's element type into
+ * *bias_dtype (may be NULL; I8_DTYPE_F16 when the image has no bias). */
+i8_status int8_layer_unpack_header_ex(const void* buf, size_t bytes, int64_t* N, int64_t* K, int* has_bias,
+                                      int* bias_dtype);
 
 /* ---------------------------------------------------------------------------
  * Inspection entry points (used by the parity tests; not needed for inference)
@@ -274,7 +286,6 @@ uint32_t int8_outlier_threshold_bits(float threshold);
  * even).  The int8 stages and the fp32 arithmetic are those of the fp16 path.
  * Any other dtype value is I8_ERR_INVALID_ARG.
  * ------------------------------------------------------------------------- */
-enum { I8_DTYPE_F16 = 0, I8_DTYPE_BF16 = 1 };
 
 /* int8_quantize_weight with W of element type `dtype`. */
 i8_status int8_quantize_weight_ex(const void* W, int dtype, int64_t N, int64_t K, int8_t* CB, float* SCB,

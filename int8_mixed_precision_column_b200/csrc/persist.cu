@@ -8,10 +8,11 @@
 //   offset  0  char[8]   magic "I8MPLYR1"
 //   offset  8  int64     N (output features)
 //   offset 16  int64     K (input features)
-//   offset 24  uint32    flags (bit 0: a bias follows SCB)
+//   offset 24  uint32    flags (bit 0: a bias follows SCB; bit 1: the bias is
+//                        bf16, else fp16)
 //   offset 28  uint32    reserved (0)
 //   offset 32  float32   SCB[N]
-//   then       fp16      bias[N]            (only when flags bit 0 is set)
+//   then       16-bit    bias[N]            (only when flags bit 0 is set)
 //   then       int8      CB[N*K], row-major
 #include <cstring>
 
@@ -40,16 +41,17 @@ size_t int8_layer_packed_bytes(int64_t N, int64_t K, int has_bias) {
   return packed_bytes(N, K, has_bias != 0);
 }
 
-i8_status int8_layer_pack(const int8_t* CB, const float* SCB, const void* bias, int64_t N, int64_t K, void* out,
-                          size_t out_bytes) {
+i8_status int8_layer_pack_ex(const int8_t* CB, const float* SCB, const void* bias, int bias_dtype, int64_t N,
+                             int64_t K, void* out, size_t out_bytes) {
   if (!shape_ok(N, K) || CB == nullptr || SCB == nullptr || out == nullptr) return I8_ERR_INVALID_ARG;
+  if (bias_dtype != I8_DTYPE_F16 && bias_dtype != I8_DTYPE_BF16) return I8_ERR_INVALID_ARG;
   const bool has_bias = bias != nullptr;
   if (out_bytes < packed_bytes(N, K, has_bias)) return I8_ERR_WORKSPACE;
   uint8_t* o = static_cast<uint8_t*>(out);
   std::memcpy(o, kMagic, 8);
   std::memcpy(o + 8, &N, 8);
   std::memcpy(o + 16, &K, 8);
-  const uint32_t flags = has_bias ? 1u : 0u, reserved = 0;
+  const uint32_t flags = has_bias ? (1u | (bias_dtype == I8_DTYPE_BF16 ? 2u : 0u)) : 0u, reserved = 0;
   std::memcpy(o + 24, &flags, 4);
   std::memcpy(o + 28, &reserved, 4);
   size_t off = kHeader;
@@ -63,7 +65,13 @@ i8_status int8_layer_pack(const int8_t* CB, const float* SCB, const void* bias, 
   return I8_OK;
 }
 
-i8_status int8_layer_unpack_header(const void* buf, size_t bytes, int64_t* N, int64_t* K, int* has_bias) {
+i8_status int8_layer_pack(const int8_t* CB, const float* SCB, const void* bias, int64_t N, int64_t K, void* out,
+                          size_t out_bytes) {
+  return int8_layer_pack_ex(CB, SCB, bias, I8_DTYPE_F16, N, K, out, out_bytes);
+}
+
+i8_status int8_layer_unpack_header_ex(const void* buf, size_t bytes, int64_t* N, int64_t* K, int* has_bias,
+                                      int* bias_dtype) {
   if (buf == nullptr || bytes < kHeader || N == nullptr || K == nullptr || has_bias == nullptr)
     return I8_ERR_INVALID_ARG;
   const uint8_t* b = static_cast<const uint8_t*>(buf);
@@ -74,12 +82,17 @@ i8_status int8_layer_unpack_header(const void* buf, size_t bytes, int64_t* N, in
   std::memcpy(&k, b + 16, 8);
   std::memcpy(&flags, b + 24, 4);
   std::memcpy(&reserved, b + 28, 4);
-  if (!shape_ok(n, k) || (flags & ~1u) != 0 || reserved != 0) return I8_ERR_INVALID_ARG;
+  if (!shape_ok(n, k) || (flags & ~3u) != 0 || flags == 2u || reserved != 0) return I8_ERR_INVALID_ARG;
   if (bytes < packed_bytes(n, k, (flags & 1u) != 0)) return I8_ERR_INVALID_ARG;
   *N = n;
   *K = k;
   *has_bias = static_cast<int>(flags & 1u);
+  if (bias_dtype != nullptr) *bias_dtype = (flags & 2u) ? I8_DTYPE_BF16 : I8_DTYPE_F16;
   return I8_OK;
+}
+
+i8_status int8_layer_unpack_header(const void* buf, size_t bytes, int64_t* N, int64_t* K, int* has_bias) {
+  return int8_layer_unpack_header_ex(buf, bytes, N, K, has_bias, nullptr);
 }
 
 i8_status int8_layer_unpack(const void* buf, size_t bytes, int8_t* CB, float* SCB, void* bias) {

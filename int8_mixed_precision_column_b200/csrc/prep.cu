@@ -285,6 +285,13 @@ __device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, in
   const uint32_t mw = kShared ? mask[chunk >> 2] : __ldg(&mask[chunk >> 2]);
   const uint32_t base = kShared ? prefix[chunk >> 2] : __ldg(&prefix[chunk >> 2]);
   const int sh = static_cast<int>(chunk & 3) * 8;
+  const uint32_t first = base + __popc(mw & ((1u << sh) - 1u));
+  if (mb == 0xffu && (first & 7u) == 0) {
+    // all 8 columns are outliers and their ranks start on a 16-byte boundary
+    // of the row (ldo is a multiple of 64): one vector store
+    *reinterpret_cast<uint4*>(xo_row + first) = v;
+    return;
+  }
   #pragma unroll
   for (int e = 0; e < 8; ++e)
     if ((mb >> e) & 1u) xo_row[base + __popc(mw & ((1u << (sh + e)) - 1u))] = h[e];

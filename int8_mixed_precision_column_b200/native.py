@@ -69,6 +69,9 @@ SIGNATURES = {
     "int8_layer_unpack_header": (_I32, [_P, _SZ, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
                                         ctypes.POINTER(ctypes.c_int)]),
     "int8_layer_unpack": (_I32, [_P, _SZ, _P, _P, _P]),
+    "int8_layer_pack_ex": (_I32, [_P, _P, _P, _I32, _I64, _I64, _P, _SZ]),
+    "int8_layer_unpack_header_ex": (_I32, [_P, _SZ, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                                           ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "int8_linear_forward_decode_static": (_I32, [_P, _I64, _I64, _P, _P, _P, _I64, _F32, _P, _P, _P, _P]),
     "int8_quantize_weight_ex": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P]),
     "int8_linear_forward_ex": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _I64, _F32, _P, _P, _P, _P, _SZ, _I32,
@@ -381,29 +384,33 @@ def workspace_views(workspace: torch.Tensor, T: int, K: int, N: int, dtype: torc
 # ---------------------------------------------------------------------------
 
 def int8_layer_pack(CB: torch.Tensor, SCB: torch.Tensor, bias: torch.Tensor | None = None) -> bytes:
-    """Byte image of a quantised layer (CB, SCB, optional bias), any device."""
+    """Byte image of a quantised layer (CB, SCB, optional fp16 or bf16 bias), any device."""
     N, K = CB.shape
     cb = CB.detach().to("cpu").contiguous()
     scb = SCB.detach().to("cpu", torch.float32).contiguous()
-    b = None if bias is None else bias.detach().to("cpu", torch.float16).contiguous()
+    bdt = torch.bfloat16 if (bias is not None and bias.dtype == torch.bfloat16) else torch.float16
+    b = None if bias is None else bias.detach().to("cpu", bdt).contiguous()
     n = int(lib().int8_layer_packed_bytes(N, K, 0 if b is None else 1))
     if n == 0:
         raise ValueError(f"unsupported shape N={N} K={K}")
     out = ctypes.create_string_buffer(n)
-    _check("int8_layer_pack", lib().int8_layer_pack(cb.data_ptr(), scb.data_ptr(), None if b is None else b.data_ptr(),
-                                                    N, K, ctypes.addressof(out), n))
+    _check("int8_layer_pack", lib().int8_layer_pack_ex(cb.data_ptr(), scb.data_ptr(),
+                                                       None if b is None else b.data_ptr(), _DTYPES[bdt], N, K,
+                                                       ctypes.addressof(out), n))
     return out.raw
 
 
 def int8_layer_unpack(image: bytes, device="cuda"):
-    """(CB int8 [N,K], SCB fp32 [N], bias fp16 [N] or None) from a byte image."""
+    """(CB int8 [N,K], SCB fp32 [N], bias fp16/bf16 [N] or None) from a byte image."""
     buf = ctypes.create_string_buffer(bytes(image), len(image))
-    N, K, hb = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int(0)
-    _check("int8_layer_unpack_header", lib().int8_layer_unpack_header(ctypes.addressof(buf), len(image),
-                                                                      ctypes.byref(N), ctypes.byref(K), ctypes.byref(hb)))
+    N, K, hb, bdt = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check("int8_layer_unpack_header", lib().int8_layer_unpack_header_ex(ctypes.addressof(buf), len(image),
+                                                                         ctypes.byref(N), ctypes.byref(K),
+                                                                         ctypes.byref(hb), ctypes.byref(bdt)))
     CB = torch.empty((N.value, K.value), dtype=torch.int8)
     SCB = torch.empty((N.value,), dtype=torch.float32)
-    b = torch.empty((N.value,), dtype=torch.float16) if hb.value else None
+    b_dtype = torch.bfloat16 if bdt.value == I8_DTYPE_BF16 else torch.float16
+    b = torch.empty((N.value,), dtype=b_dtype) if hb.value else None
     _check("int8_layer_unpack", lib().int8_layer_unpack(ctypes.addressof(buf), len(image), CB.data_ptr(), SCB.data_ptr(),
                                                         None if b is None else b.data_ptr()))
     return CB.to(device), SCB.to(device), (None if b is None else b.to(device))

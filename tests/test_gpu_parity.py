@@ -140,6 +140,18 @@ def test_ragged_tensor_core(T, K, N, planted, thr, path):
     check_forward(p, gpu_forward(p, path))
 
 
+@pytest.mark.parametrize("T,K,N,planted,path", [
+    (300, 20480, 256, 9, "tc"),       # K > 16384, few rows: two-pass CTA-per-row quantisation
+    (2048, 20480, 128, 9, "tc"),      # K > 16384, many rows: warp-per-row quantisation
+    (40, 131072, 64, 33, "tc"),       # the largest K the library takes
+    (16, 131072, 64, 33, "decode"),   # ... through the one-kernel decode prep
+    (3, 131072, 48, 2, "auto"),
+])
+def test_long_rows_and_maximum_k(T, K, N, planted, path):
+    p = workloads.make_problem("longk", T, K, N, n_planted=planted, bias_std=0.01, seed=T + K)
+    check_forward(p, gpu_forward(p, path), check_wo=path != "decode" and not (path == "auto" and T <= 16))
+
+
 @pytest.mark.parametrize("T", [1, 2, 5, 8, 9, 15, 16])
 def test_decode_matches_oracle_and_tensor_core(T):
     p = workloads.make_problem("dec", T, 1216, 400 - 400 % 16, n_planted=5, bias_std=0.01, seed=T)

@@ -47,6 +47,21 @@ def test_byte_layout_is_the_documented_one():
     assert len(img) == native.lib().int8_layer_packed_bytes(16, 32, 1) == 32 + 64 + 32 + 512
 
 
+def test_bf16_bias_round_trip_and_flag():
+    CB, SCB, bias = _layer(N=32, K=48, seed=2)
+    b16 = bias.float().mul(3.0).to(torch.bfloat16)
+    img = native.int8_layer_pack(CB, SCB, b16)
+    assert struct.unpack_from("<qqII", img, 8) == (32, 48, 3, 0)     # bias present, bf16
+    cb2, scb2, b2 = native.int8_layer_unpack(img, device="cpu")
+    assert b2.dtype == torch.bfloat16 and torch.equal(b2, b16)
+    assert torch.equal(cb2, CB) and torch.equal(scb2, SCB)
+    # the fp16 image of the same layer records no bf16 flag
+    assert struct.unpack_from("<I", native.int8_layer_pack(CB, SCB, bias), 24) == (1,)
+    for flags in (4, 2 | 4, 8):
+        with pytest.raises(native.Int8mpError):
+            native.int8_layer_unpack(img[:24] + struct.pack("<I", flags) + img[28:], device="cpu")
+
+
 def test_malformed_images_are_rejected():
     CB, SCB, bias = _layer()
     img = native.int8_layer_pack(CB, SCB, bias)
