@@ -287,7 +287,7 @@ def run_sharded(args, rank, world, local_rank) -> dict | None:
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS", "frac": achieved / peak,
                      "traffic": None, "traffic_source": "whole sharded forward per rank (3 kernels + 2 barriers)",
                      "kernel": "whole forward", "peak_source": f"{peak_src} bf16_tflops (burst) x {INT8_PER_BF16}"},
-        "gpu_launches": (3 if p.threshold > 0 else 2) * args.steps,
+        "gpu_launches": (2 if T <= 16 else (3 if p.threshold > 0 else 2)) * args.steps,
         "clocks": clocks, "e2e": None, "device": torch.cuda.get_device_name(dev),
     }
 
@@ -506,7 +506,9 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
                 "algorithmic_ops_per_launch": work["int8_ops"], "fp16_flops_per_launch": work["fp16_flops"],
                 "achieved_counts": "int8 ops + 2 x 16-bit outlier flops (int8-equivalent tensor work)",
                 "ms_per_launch": prod_avg}
-    launches_per_step = 3 if p.threshold > 0 else 2
+    # kernels per forward: decode = the one-kernel prep + the GEMV; otherwise
+    # outlier pass (only with a threshold) + row quantisation + product
+    launches_per_step = 2 if decode else (3 if p.threshold > 0 else 2)
     tops, tok_s = whole_job(work["int8_ops"], T, world, ms_per_step)
     out = {
         "metric": METRIC,
