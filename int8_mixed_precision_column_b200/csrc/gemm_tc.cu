@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int num_n = static_cast<int>((p.N + BN - 1) / BN);
   const int num_tiles = num_m * num_n;
   griddep_wait();  // n_out and the operands come from the preceding kernels
-  const int n_out = (p.n_out != nullptr) ? *p.n_out : 0;
+  const int n_out = (p.n_out != nullptr) ? __ldcg(p.n_out) : 0;
   const int nkb_o = (p.mode == 0) ? (n_out + 63) / 64 : 0;
   const int nkb = p.nkb_i8 + nkb_o;
   const bool has_out = nkb_o > 0;

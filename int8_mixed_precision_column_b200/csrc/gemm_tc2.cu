@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   // The set-up above overlaps the tail of the row quantisation (programmatic
   // launch); n_out and every operand are read only after it has completed.
   griddep_wait();
-  const int n_out = (p.n_out != nullptr && p.mode == 0) ? *p.n_out : 0;
+  const int n_out = (p.n_out != nullptr && p.mode == 0) ? __ldcg(p.n_out) : 0;
   const int nkb_o = (n_out + 63) / 64;
   const int nkb = p.nkb_i8 + nkb_o;
   const bool has_out = nkb_o > 0;                            // outliers on tensor cores (fp32 TMEM)

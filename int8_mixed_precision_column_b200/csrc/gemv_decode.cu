@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
   if (threadIdx.x < kPrefetchRows && g_begin * 8 + threadIdx.x < g_end * 8)
     prefetch_l2(p.CB + (g_begin * 8 + threadIdx.x) * p.K, static_cast<uint32_t>(p.K));
   griddep_wait();
-  const int n_out = (p.mode == 0) ? *p.n_out : 0;
+  const int n_out = (p.mode == 0) ? __ldcg(p.n_out) : 0;
   const bool row_a = g < p.T;
   const bool row_b = g + 8 < p.T;
   const int8_t* xa_base = p.Xq + static_cast<int64_t>(g) * p.K + t4 * 16;
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
         const int64_t j = g0 * 8 + r;
         float wv = 0.0f;
         if (j < g_end * 8) {
-          const int64_t col = __ldg(&p.idx[ob + o]);
+          const int64_t col = __ldcg(&p.idx[ob + o]);
           if (p.Wf != nullptr) {
             wv = E::to_float(static_cast<const TE*>(p.Wf)[j * p.K + col]);
           } else {

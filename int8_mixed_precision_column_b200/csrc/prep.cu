@@ -196,10 +196,16 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const TE* __
 cudaError_t launch_outliers(const void* X, int dtype, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
                             uint32_t* prefix, int32_t* idx, int32_t* n_out, DevStatus* st, cudaStream_t s) {
   // The 8 warps split the rows (measured faster than warps side by side along
-  // the columns, which gives fewer, longer-lived CTAs).
+  // the columns, which gives fewer, longer-lived CTAs).  128 rows per CTA,
+  // fewer (down to 32) while the grid would hold under 4 CTAs per SM.
   const int wc = 1;
-  const int64_t rows_per_cta = 128;
   const int64_t slabs = (K + 256 * wc - 1) / (256 * wc);
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t rows_per_cta = 128;
+  while (rows_per_cta > 32 && slabs * ((T + rows_per_cta - 1) / rows_per_cta) < 4 * static_cast<int64_t>(sms))
+    rows_per_cta /= 2;
   const int64_t chunks = (T + rows_per_cta - 1) / rows_per_cta;
   if (slabs > 0x7fffffff || chunks > 65535) return cudaErrorInvalidValue;
   dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(chunks));
@@ -234,8 +240,11 @@ constexpr int kRowThreads = 256;
 constexpr int kRowWarps = kRowThreads / 32;
 constexpr int kRowUnroll = 8;
 
+// The outlier pass's outputs (mask, prefix, idx, n_out) decide addresses in the
+// kernels that follow it under programmatic launch: those kernels read them
+// through L2 (ld.global.cg), never through the non-coherent read-only path.
 __device__ __forceinline__ uint32_t mask_byte(const uint32_t* mask, int64_t chunk) {
-  return (__ldg(&mask[chunk >> 2]) >> ((chunk & 3) * 8)) & 0xffu;
+  return (__ldcg(&mask[chunk >> 2]) >> ((chunk & 3) * 8)) & 0xffu;
 }
 
 // Largest magnitude pattern among the non-outlier elements of a chunk.
@@ -282,8 +291,8 @@ template <typename TE, bool kShared = false>
 __device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, int64_t chunk, const uint32_t* mask,
                                                  const uint32_t* prefix, TE* xo_row) {
   const TE* h = reinterpret_cast<const TE*>(&v);
-  const uint32_t mw = kShared ? mask[chunk >> 2] : __ldg(&mask[chunk >> 2]);
-  const uint32_t base = kShared ? prefix[chunk >> 2] : __ldg(&prefix[chunk >> 2]);
+  const uint32_t mw = kShared ? mask[chunk >> 2] : __ldcg(&mask[chunk >> 2]);
+  const uint32_t base = kShared ? prefix[chunk >> 2] : __ldcg(&prefix[chunk >> 2]);
   const int sh = static_cast<int>(chunk & 3) * 8;
   const uint32_t first = base + __popc(mw & ((1u << sh) - 1u));
   if (mb == 0xffu && (first & 7u) == 0) {
@@ -335,7 +344,7 @@ __device__ __forceinline__ void wo_gather(int64_t wblk, int64_t wo_blocks, int n
           const int o = o0 + i + h;
           f[h] = 0.0f;
           if (o < n_out) {
-            const int col = __ldg(&idx[o]);
+            const int col = __ldcg(&idx[o]);
             f[h] = wfrow != nullptr ? E::to_float(wfrow[col])
                                     : __fdiv_rn(__fmul_rn(static_cast<float>(__ldg(&cbrow[col])), scb), 127.0f);
           }
@@ -358,7 +367,7 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
   const int lane = threadIdx.x & 31;
   griddep_launch_dependents();
   griddep_wait();  // mask, prefix, idx, n_out come from the outlier pass
-  const int n_out = *n_out_p;
+  const int n_out = __ldcg(n_out_p);
   const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
 
   if (static_cast<int64_t>(blockIdx.x) >= row_blocks) {
@@ -423,70 +432,80 @@ constexpr int kRowCtaThreads = 256;
 constexpr int kRowCtaUnroll = 8;
 constexpr int64_t kResidentMaxK = static_cast<int64_t>(kRowCtaThreads) * kRowCtaUnroll * 8;
 
+// A CTA takes R = 2^rpc_log rows (1, 2, 4 or 8), S = 256 / R threads per row:
+// short rows share a CTA, so that every thread still has up to 8 loads in
+// flight (R > 1 only when the row fits the S threads x 8 chunks).
 template <typename TE, bool kResident>
 __global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
     const TE* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
     const uint32_t* __restrict__ prefix, const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p,
     int8_t* __restrict__ Xq, float* __restrict__ sA, TE* __restrict__ Xo, int64_t ldo,
     const int8_t* __restrict__ CB, const float* __restrict__ SCB, int64_t N, TE* __restrict__ Wo,
-    const TE* __restrict__ Wf, int64_t row_blocks, int64_t wo_blocks) {
+    const TE* __restrict__ Wf, int64_t row_blocks, int64_t wo_blocks, int rpc_log) {
   using E = Elem<TE>;
   __shared__ uint32_t s_max[kRowCtaThreads / 32];
   griddep_launch_dependents();
   griddep_wait();  // mask, prefix, idx, n_out come from the outlier pass
-  const int n_out = *n_out_p;
+  const int n_out = __ldcg(n_out_p);
   const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
   if (static_cast<int64_t>(blockIdx.x) >= row_blocks) {
     wo_gather<TE, kRowCtaThreads>(static_cast<int64_t>(blockIdx.x) - row_blocks, wo_blocks, n_out, npad, idx, CB,
                                   SCB, N, K, Wo, ldo, Wf);
     return;
   }
-  const int64_t t = blockIdx.x;
+  const int S = kRowCtaThreads >> rpc_log;  // threads per row, a multiple of 32
+  const int sub = static_cast<int>(threadIdx.x) / S;
+  const int tid = static_cast<int>(threadIdx.x) - sub * S;
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) << rpc_log) + sub;
+  const bool live = t < T;   // whole warps share a row, so `live` is warp-uniform
   const int64_t nv = K / 8;
   const uint4* src = reinterpret_cast<const uint4*>(X + t * K);
-  constexpr int64_t kStep = static_cast<int64_t>(kRowCtaThreads) * kRowCtaUnroll;
+  const int64_t step = static_cast<int64_t>(S) * kRowCtaUnroll;
   uint32_t mmax = 0;
   uint4 v[kRowCtaUnroll];   // with kResident: the whole row share of this thread
   uint32_t mbs[kRowCtaUnroll];
-  for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
-    #pragma unroll
-    for (int u = 0; u < kRowCtaUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
-      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-      mbs[u] = (c < nv) ? mask_byte(mask, c) : 0u;
+  if (live) {
+    for (int64_t c0 = tid; c0 < nv; c0 += step) {
+      #pragma unroll
+      for (int u = 0; u < kRowCtaUnroll; ++u) {
+        const int64_t c = c0 + static_cast<int64_t>(S) * u;
+        v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+        mbs[u] = (c < nv) ? mask_byte(mask, c) : 0u;
+      }
+      #pragma unroll
+      for (int u = 0; u < kRowCtaUnroll; ++u) {
+        const int64_t c = c0 + static_cast<int64_t>(S) * u;
+        if (c < nv) mmax = max(mmax, chunk_max_mag_kept<TE>(v[u], mbs[u]));
+      }
+      if constexpr (kResident) break;
     }
-    #pragma unroll
-    for (int u = 0; u < kRowCtaUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
-      if (c < nv) mmax = max(mmax, chunk_max_mag_kept<TE>(v[u], mbs[u]));
-    }
-    if constexpr (kResident) break;
   }
   #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
   if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = mmax;
   __syncthreads();
+  if (!live) return;
   mmax = 0;
-  #pragma unroll
-  for (int w = 0; w < kRowCtaThreads / 32; ++w) mmax = max(mmax, s_max[w]);
+  const int w0 = sub * (S / 32);
+  for (int w = w0; w < w0 + S / 32; ++w) mmax = max(mmax, s_max[w]);
   const float absmax = E::mag_to_float(mmax);
   const float inv = scale_inv(absmax);
-  if (threadIdx.x == 0) sA[t] = absmax;
+  if (tid == 0) sA[t] = absmax;
 
   uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
   TE* xo_row = Xo + t * ldo;
-  for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
+  for (int64_t c0 = tid; c0 < nv; c0 += step) {
     if constexpr (!kResident) {
       #pragma unroll
       for (int u = 0; u < kRowCtaUnroll; ++u) {
-        const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+        const int64_t c = c0 + static_cast<int64_t>(S) * u;
         v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
         mbs[u] = (c < nv) ? mask_byte(mask, c) : 0u;
       }
     }
     #pragma unroll
     for (int u = 0; u < kRowCtaUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kRowCtaThreads) * u;
+      const int64_t c = c0 + static_cast<int64_t>(S) * u;
       if (c < nv) {
         dst[c] = row_codes_fast<TE>(v[u], mbs[u], inv);
         if (mbs[u]) scatter_outliers<TE>(v[u], mbs[u], c, mask, prefix, xo_row);
@@ -494,7 +513,7 @@ __global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
     }
     if constexpr (kResident) break;
   }
-  for (int64_t o = n_out + threadIdx.x; o < npad; o += kRowCtaThreads) xo_row[o] = E::from_float(0.0f);
+  for (int64_t o = n_out + tid; o < npad; o += S) xo_row[o] = E::from_float(0.0f);
 }
 
 // ---------------------------------------------------------------------------
@@ -651,17 +670,21 @@ cudaError_t launch_prep_small(const void* X, int dtype, int64_t T, int64_t K, ui
 }
 
 template <typename TE>
-static cudaError_t launch_rowquant_t(const cudaLaunchConfig_t& cfg, bool cta_rows, bool resident, const void* X,
-                                     int64_t T,
-                                     int64_t K, const uint32_t* mask, const uint32_t* prefix, const int32_t* idx,
-                                     const int32_t* n_out, int8_t* Xq, float* sA, void* Xo, int64_t ldo,
-                                     const int8_t* CB, const float* SCB, int64_t N, void* Wo, const void* Wf,
-                                     int64_t row_blocks, int64_t wo_blocks) {
-  return cudaLaunchKernelEx(&cfg,
-                            cta_rows ? (resident ? rowquant_cta_kernel<TE, true> : rowquant_cta_kernel<TE, false>)
-                                     : rowquant_kernel<TE>,
-                            static_cast<const TE*>(X), T, K, mask, prefix, idx, n_out, Xq, sA, static_cast<TE*>(Xo),
-                            ldo, CB, SCB, N, static_cast<TE*>(Wo), static_cast<const TE*>(Wf), row_blocks, wo_blocks);
+static cudaError_t launch_rowquant_t(const cudaLaunchConfig_t& cfg, bool cta_rows, bool resident, int rpc_log,
+                                     const void* X, int64_t T, int64_t K, const uint32_t* mask,
+                                     const uint32_t* prefix, const int32_t* idx, const int32_t* n_out, int8_t* Xq,
+                                     float* sA, void* Xo, int64_t ldo, const int8_t* CB, const float* SCB, int64_t N,
+                                     void* Wo, const void* Wf, int64_t row_blocks, int64_t wo_blocks) {
+  const TE* x = static_cast<const TE*>(X);
+  TE* xo = static_cast<TE*>(Xo);
+  TE* wo = static_cast<TE*>(Wo);
+  const TE* wf = static_cast<const TE*>(Wf);
+  if (!cta_rows)
+    return cudaLaunchKernelEx(&cfg, rowquant_kernel<TE>, x, T, K, mask, prefix, idx, n_out, Xq, sA, xo, ldo, CB, SCB, N,
+                              wo, wf, row_blocks, wo_blocks);
+  return cudaLaunchKernelEx(&cfg, resident ? rowquant_cta_kernel<TE, true> : rowquant_cta_kernel<TE, false>, x, T, K,
+                            mask, prefix, idx, n_out, Xq, sA, xo, ldo, CB, SCB, N, wo, wf, row_blocks, wo_blocks,
+                            rpc_log);
 }
 
 cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, const uint32_t* mask,
@@ -669,11 +692,15 @@ cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, cons
                             void* Xo, int64_t ldo, const int8_t* CB, const float* SCB, int64_t N, void* Wo,
                             bool with_wo, const void* Wf, int num_sms, DevStatus* st, bool pdl, cudaStream_t s) {
   (void)st;
-  // One CTA per row with the row held in registers whenever it fits (X read
-  // once); otherwise warp-per-row CTAs while they fill the SMs, and one CTA
-  // per row (two passes) below that.
+  // CTA rows with the row held in registers whenever it fits (X read once),
+  // several short rows to a CTA; otherwise warp-per-row CTAs while they fill
+  // the SMs, and one CTA per row (two passes) below that.
+  const int64_t nv = K / 8;
   const bool resident = K <= kResidentMaxK;
   const bool cta_rows = resident || (T + kRowWarps - 1) / kRowWarps < num_sms;
+  int rpc_log = 0;
+  if (resident)
+    while (rpc_log < 3 && nv * (int64_t(2) << rpc_log) <= int64_t(kRowCtaThreads) * kRowCtaUnroll) ++rpc_log;
   const int threads = cta_rows ? kRowCtaThreads : kRowThreads;
   int64_t wo_blocks = 0;
   if (with_wo) {
@@ -682,7 +709,8 @@ cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, cons
     if (wo_blocks > cap) wo_blocks = cap;
     if (wo_blocks < 1) wo_blocks = 1;
   }
-  const int64_t row_blocks = cta_rows ? T : (T + kRowWarps - 1) / kRowWarps;
+  const int64_t row_blocks =
+      cta_rows ? (T + (int64_t(1) << rpc_log) - 1) >> rpc_log : (T + kRowWarps - 1) / kRowWarps;
   const int64_t blocks = row_blocks + wo_blocks;
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
@@ -696,10 +724,10 @@ cudaError_t launch_rowquant(const void* X, int dtype, int64_t T, int64_t K, cons
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   if (dtype == kBF16)
-    return launch_rowquant_t<__nv_bfloat16>(cfg, cta_rows, resident, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB,
-                                            SCB, N, Wo, Wf, row_blocks, wo_blocks);
-  return launch_rowquant_t<__half>(cfg, cta_rows, resident, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, ldo, CB, SCB, N,
-                                   Wo, Wf, row_blocks, wo_blocks);
+    return launch_rowquant_t<__nv_bfloat16>(cfg, cta_rows, resident, rpc_log, X, T, K, mask, prefix, idx, n_out, Xq,
+                                            sA, Xo, ldo, CB, SCB, N, Wo, Wf, row_blocks, wo_blocks);
+  return launch_rowquant_t<__half>(cfg, cta_rows, resident, rpc_log, X, T, K, mask, prefix, idx, n_out, Xq, sA, Xo,
+                                   ldo, CB, SCB, N, Wo, Wf, row_blocks, wo_blocks);
 }
 
 }  // namespace i8mp

@@ -132,7 +132,9 @@ class NShardedLinear:
         return g.group_name
 
     def forward(self, X: torch.Tensor, threshold: float) -> torch.Tensor:
-        """Y [T, N] (the full output, identical on every rank)."""
+        """Y [T, N] (the full output, identical on every rank).  In peer mode the
+        result is a view of the layer's symmetric output buffer: the next
+        forward overwrites it (clone it to keep it)."""
         T = X.shape[0]
         if T > self.T_max:
             raise ValueError(f"T={T} > T_max={self.T_max}")
