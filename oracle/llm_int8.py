@@ -23,7 +23,7 @@ It restates, step by step and in plain numpy, what the pages describe:
   scheme: separate normalisation constants per inner product; outlier
   feature dimensions go to a second 16-bit matmul.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 threshold <= 0 disables the decomposition; "exceeds" is strict ``>``;
 a column is an outlier for every token if any token exceeds; the row absmax
 runs over non-outlier columns only; rounding is half away from zero after an
