@@ -244,32 +244,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const float ra = (row_ok && p.mode == 0) ? __ldg(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
       #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        const int col0 = half * 128 + c * 16;
+      for (int c = 0; c < 4; ++c) {
+        const int col0 = half * 128 + c * 32;
         const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
-        uint32_t acc[16];
-        uint32_t fo[16];  // fp32 outlier product (when the tile has outlier columns)
-        tmem_ld_32x32b_x16(tmem_base + lane_base + static_cast<uint32_t>(buf) * 256u + col0, acc);
-        if (has_out) tmem_ld_32x32b_x16(tmem_base + lane_base + 256u + col0, fo);
+        uint32_t acc[32];
+        uint32_t fo[32];
+        tmem_ld_32x32b_x32(tmem_base + lane_base + static_cast<uint32_t>(buf) * 256u + col0, acc);
+        if (has_out) tmem_ld_32x32b_x32(tmem_base + lane_base + 256u + col0, fo);
         tmem_ld_wait();
         if (p.mode == 1) {
           if (row_ok) {
             int32_t* dst = p.acc_out + row * p.N + gcol0;
             #pragma unroll
-            for (int g = 0; g < 4; ++g)
+            for (int g = 0; g < 8; ++g)
               if (gcol0 + g * 4 + 4 <= p.N)
                 reinterpret_cast<int4*>(dst)[g] = make_int4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]);
           }
           continue;
         }
-        // column scales and bias of these 16 columns: every lane reads the same
-        // addresses, so the loads are L1 broadcasts
-        float sc[16], bi[16];
-        const bool full = gcol0 + 16 <= p.N;
+        float sc[32], bi[32];
+        const bool full = gcol0 + 32 <= p.N;
         if (full && p.vec_scb) {
           const float4* s4 = reinterpret_cast<const float4*>(p.SCB + gcol0);
           #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
+          for (int q4 = 0; q4 < 8; ++q4) {
             const float4 v = __ldg(s4 + q4);
             sc[4 * q4] = v.x;
             sc[4 * q4 + 1] = v.y;
@@ -278,15 +276,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         } else {
           #pragma unroll
-          for (int i = 0; i < 16; ++i) sc[i] = (gcol0 + i < p.N) ? __ldg(&p.SCB[gcol0 + i]) : 0.0f;
+          for (int i = 0; i < 32; ++i) sc[i] = (gcol0 + i < p.N) ? __ldg(&p.SCB[gcol0 + i]) : 0.0f;
         }
         if (p.bias == nullptr) {
           #pragma unroll
-          for (int i = 0; i < 16; ++i) bi[i] = 0.0f;
+          for (int i = 0; i < 32; ++i) bi[i] = 0.0f;
         } else if (full && p.vec_bias) {
           const uint4* b8 = reinterpret_cast<const uint4*>(static_cast<const TE*>(p.bias) + gcol0);
           #pragma unroll
-          for (int q8 = 0; q8 < 2; ++q8) {
+          for (int q8 = 0; q8 < 4; ++q8) {
             const uint4 v = __ldg(b8 + q8);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             #pragma unroll
@@ -298,12 +296,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         } else {
           #pragma unroll
-          for (int i = 0; i < 16; ++i)
+          for (int i = 0; i < 32; ++i)
             bi[i] = (gcol0 + i < p.N) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[gcol0 + i]) : 0.0f;
         }
-        uint32_t packed[8];
+        uint32_t packed[16];
         #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
+        for (int i = 0; i < 32; i += 2) {
           float y0 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i])), ra * sc[i], bi[i]);
           float y1 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i + 1])), ra * sc[i + 1], bi[i + 1]);
           if (has_out) {
@@ -316,7 +314,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int64_t off = row * p.yd.ld + gcol0;
           TE* dst = static_cast<TE*>(p.Y) + off;
           #pragma unroll
-          for (int g = 0; g < 2; ++g)
+          for (int g = 0; g < 4; ++g)
             if (gcol0 + g * 8 + 8 <= p.N) {
               const uint4 v = make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
               reinterpret_cast<uint4*>(dst)[g] = v;
