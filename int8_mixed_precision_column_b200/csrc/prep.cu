@@ -529,7 +529,10 @@ constexpr int kSmallMaxK = 131072;
 constexpr int kSmallThreads = 512;
 constexpr int kSmallUnroll = 4;
 
-template <typename TE>
+// kResident (K <= 512 x 4 x 8): each thread keeps its 4 chunks of the CTA's own
+// row in registers from the first load to the codes; other rows are read for
+// the mask only.
+template <typename TE, bool kResident>
 __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
     const TE* __restrict__ X, int64_t T, int64_t K, uint32_t hbits, uint32_t* __restrict__ mask,
     uint32_t* __restrict__ prefix, int32_t* __restrict__ idx, int32_t* __restrict__ n_out_p, int8_t* __restrict__ Xq,
@@ -544,10 +547,37 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
   const int64_t nw = (K + 31) / 32;
   const bool on = hbits != 0xffffffffu;
   const uint32_t h2 = hbits | (hbits << 16);
+  const int64_t t = blockIdx.x;
+  const uint4* src = reinterpret_cast<const uint4*>(X + t * K);
+  uint4 v[kSmallUnroll];  // with kResident: this thread's chunks of row t
+  if constexpr (kResident) {
+    #pragma unroll
+    for (int u = 0; u < kSmallUnroll; ++u) {
+      const int64_t c = threadIdx.x + static_cast<int64_t>(kSmallThreads) * u;
+      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+  }
   for (int64_t w = threadIdx.x; w < nw; w += kSmallThreads) s_mask[w] = 0;
   __syncthreads();
   // mask: column chunk c is flagged from all T rows
-  if (on) {
+  if (on && kResident) {
+    #pragma unroll
+    for (int u = 0; u < kSmallUnroll; ++u) {
+      const int64_t c = threadIdx.x + static_cast<int64_t>(kSmallThreads) * u;
+      if (c >= nv) continue;
+      uint32_t bits = flag_bits8<TE>(v[u], h2);
+      for (int64_t r = 0; r < T; r += 4) {
+        uint4 o[4];
+        #pragma unroll
+        for (int q = 0; q < 4; ++q)
+          o[q] = (r + q < T && r + q != t) ? __ldg(reinterpret_cast<const uint4*>(X + (r + q) * K) + c)
+                                           : make_uint4(0, 0, 0, 0);
+        #pragma unroll
+        for (int q = 0; q < 4; ++q) bits |= flag_bits8<TE>(o[q], h2);
+      }
+      if (bits) atomicOr(&s_mask[c >> 2], bits << ((c & 3) * 8));
+    }
+  } else if (on) {
     for (int64_t c = threadIdx.x; c < nv; c += kSmallThreads) {
       uint32_t bits = 0;
       int64_t r = 0;
@@ -602,24 +632,24 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
   __syncthreads();
 
   // this CTA's row, as rowquant_cta_kernel with the mask from shared memory
-  const int64_t t = blockIdx.x;
   const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
-  const uint4* src = reinterpret_cast<const uint4*>(X + t * K);
   const uint8_t* mb8 = reinterpret_cast<const uint8_t*>(s_mask);
   constexpr int64_t kStep = static_cast<int64_t>(kSmallThreads) * kSmallUnroll;
   uint32_t mmax = 0;
   for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
-    uint4 v[kSmallUnroll];
-    #pragma unroll
-    for (int u = 0; u < kSmallUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kSmallThreads) * u;
-      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    if constexpr (!kResident) {
+      #pragma unroll
+      for (int u = 0; u < kSmallUnroll; ++u) {
+        const int64_t c = c0 + static_cast<int64_t>(kSmallThreads) * u;
+        v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+      }
     }
     #pragma unroll
     for (int u = 0; u < kSmallUnroll; ++u) {
       const int64_t c = c0 + static_cast<int64_t>(kSmallThreads) * u;
       if (c < nv) mmax = max(mmax, chunk_max_mag_kept<TE>(v[u], mb8[c]));
     }
+    if constexpr (kResident) break;
   }
   #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
@@ -634,11 +664,12 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
   uint2* dst = reinterpret_cast<uint2*>(Xq + t * K);
   TE* xo_row = Xo + t * ldo;
   for (int64_t c0 = threadIdx.x; c0 < nv; c0 += kStep) {
-    uint4 v[kSmallUnroll];
-    #pragma unroll
-    for (int u = 0; u < kSmallUnroll; ++u) {
-      const int64_t c = c0 + static_cast<int64_t>(kSmallThreads) * u;
-      v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    if constexpr (!kResident) {
+      #pragma unroll
+      for (int u = 0; u < kSmallUnroll; ++u) {
+        const int64_t c = c0 + static_cast<int64_t>(kSmallThreads) * u;
+        v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+      }
     }
     #pragma unroll
     for (int u = 0; u < kSmallUnroll; ++u) {
@@ -649,6 +680,7 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
         if (mb) scatter_outliers<TE, true>(v[u], mb, c, s_mask, s_prefix, xo_row);
       }
     }
+    if constexpr (kResident) break;
   }
   for (int64_t o = n_out + threadIdx.x; o < npad; o += kSmallThreads) xo_row[o] = E::from_float(0.0f);
 }
@@ -658,14 +690,16 @@ cudaError_t launch_prep_small(const void* X, int dtype, int64_t T, int64_t K, ui
                               int64_t ldo, DevStatus* st, cudaStream_t s) {
   if (T < 1 || T > kDecodeMaxT || K > kSmallMaxK) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(T));
-  if (dtype == kBF16)
-    prep_small_kernel<__nv_bfloat16><<<grid, kSmallThreads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(X), T, K, hbits, mask, prefix, idx, n_out, Xq, sA,
-        static_cast<__nv_bfloat16*>(Xo), ldo, st);
-  else
-    prep_small_kernel<__half><<<grid, kSmallThreads, 0, s>>>(static_cast<const __half*>(X), T, K, hbits, mask,
-                                                              prefix, idx, n_out, Xq, sA, static_cast<__half*>(Xo),
-                                                              ldo, st);
+  const bool resident = K <= static_cast<int64_t>(kSmallThreads) * kSmallUnroll * 8;
+  if (dtype == kBF16) {
+    auto* k = resident ? prep_small_kernel<__nv_bfloat16, true> : prep_small_kernel<__nv_bfloat16, false>;
+    k<<<grid, kSmallThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(X), T, K, hbits, mask, prefix, idx, n_out,
+                                      Xq, sA, static_cast<__nv_bfloat16*>(Xo), ldo, st);
+  } else {
+    auto* k = resident ? prep_small_kernel<__half, true> : prep_small_kernel<__half, false>;
+    k<<<grid, kSmallThreads, 0, s>>>(static_cast<const __half*>(X), T, K, hbits, mask, prefix, idx, n_out, Xq, sA,
+                                      static_cast<__half*>(Xo), ldo, st);
+  }
   return cudaGetLastError();
 }
 
