@@ -259,29 +259,41 @@ __device__ __forceinline__ uint32_t chunk_max_mag_kept(const uint4& v, uint32_t 
   return m;
 }
 
-// Round half away from zero for |y| <= 127 * (1 + 2^-23), the range of
-// x * fp32(127/absmax) when |x| <= absmax.  For |y| >= 0.5, |y| + 0.5 is either
-// exact or rounds within the same integer interval, so truncating it gives
-// the nearest integer with ties away from zero; |y| < 0.5 gives 0.
+// Round half away from zero for y = x * fp32(127/absmax) with |x| <= absmax.
+// y + copysign(0.5, y) equals sign(y) * (|y| + 0.5) as fp32 computes it; for
+// |y| >= 0.5 that sum is exact or rounds within the same integer interval, so
+// truncating toward zero gives the nearest integer with ties away from zero.
+// For |y| < 0.5 the code is 0 (tested explicitly: just below 0.5, |y| + 0.5
+// rounds up to 1.0 in fp32).  |y| <= 127 * (1 + 2^-24)^2 < 127.5 keeps the
+// result within +-127 without a clamp.
 __device__ __forceinline__ int round_away_code(float y) {
-  const float a = fabsf(y);
-  int q = (a < 0.5f) ? 0 : __float2int_rz(a + 0.5f);
-  q = min(q, 127);
-  return (y < 0.0f) ? -q : q;
+  return (fabsf(y) < 0.5f) ? 0 : __float2int_rz(y + copysignf(0.5f, y));
 }
 
 template <typename TE>
 __device__ __forceinline__ uint2 row_codes_fast(const uint4& v, uint32_t mb, float inv) {
   const uint32_t pairs[4] = {v.x, v.y, v.z, v.w};
-  uint32_t w[2] = {0u, 0u};
+  int q[8];
   #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const float2 f = Elem<TE>::to_float2(pairs[p]);
-    const int q0 = ((mb >> (2 * p)) & 1u) ? 0 : round_away_code(__fmul_rn(f.x, inv));
-    const int q1 = ((mb >> (2 * p + 1)) & 1u) ? 0 : round_away_code(__fmul_rn(f.y, inv));
-    w[p >> 1] |= ((static_cast<uint32_t>(q0) & 0xffu) | ((static_cast<uint32_t>(q1) & 0xffu) << 8)) << (16 * (p & 1));
+    q[2 * p] = round_away_code(__fmul_rn(f.x, inv));
+    q[2 * p + 1] = round_away_code(__fmul_rn(f.y, inv));
   }
-  return make_uint2(w[0], w[1]);
+  // low bytes of the codes, 4 to a word
+  uint32_t w0 = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+  uint32_t w1 = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
+  if (mb) {  // outlier columns get code 0 (rare: a byte mask from the 8 flag bits)
+    uint32_t k0 = 0, k1 = 0;
+    #pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      k0 |= ((mb >> e) & 1u) ? (0xffu << (8 * e)) : 0u;
+      k1 |= ((mb >> (4 + e)) & 1u) ? (0xffu << (8 * e)) : 0u;
+    }
+    w0 &= ~k0;
+    w1 &= ~k1;
+  }
+  return make_uint2(w0, w1);
 }
 
 // Scatter the outlier entries of one 8-column chunk into the Xo row.  mask and
