@@ -480,7 +480,8 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     work = algorithmic_work(T, K, N, n_outliers)
     peaks, peak_src = load_peaks()
     prod_avg = statistics.mean(prod_ms)
-    decode = T <= 16 if args.path == 0 else args.path == 2
+    product = native.int8_linear_product_kernel(T, K, N, args.path)  # the kernel the forward ran
+    decode = product == native.PATH_DECODE
     traffic_key = args.workload if elem == torch.float16 else f"{args.workload}_bf16"
     if decode:
         achieved = work["product_bytes"] / (prod_avg * 1e-3) / 1e9
@@ -496,7 +497,7 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
         peak = peaks["bf16_tflops"] * INT8_PER_BF16
         equiv_ops = work["int8_ops"] + INT8_PER_BF16 * work["fp16_flops"]
         achieved = equiv_ops / (prod_avg * 1e-3) / 1e12
-        kname = "gemm_i8_tc_kernel" if args.path == 3 else "gemm_i8_tc2_kernel"
+        kname = "gemm_i8_tc_kernel" if product == native.PATH_TENSOR_CORE_1SM else "gemm_i8_tc2_kernel"
         traffic, traffic_src = recorded_traffic(kname, traffic_key)
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS",
                 "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,

@@ -101,8 +101,8 @@ size_t int8_linear_workspace_bytes(int64_t T, int64_t K, int64_t N);
  *             aligned; its contents need no initialisation and are
  *             overwritten.  One workspace must not be shared by forwards
  *             that can run concurrently.
- * T <= 16 takes the weight-streaming decode kernel, larger T the tensor-core
- * GEMM; both give the same integer stages.  Asynchronous on `stream`; n_out
+ * T <= 16 takes the weight-streaming decode kernel, larger T a tensor-core
+ * GEMM (see int8_linear_forward_path); all give the same integer stages.  Asynchronous on `stream`; n_out
  * stays on the device (no host synchronisation).
  */
 i8_status int8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
@@ -111,10 +111,12 @@ i8_status int8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t*
                               cudaStream_t stream);
 
 /* As int8_linear_forward, with the product kernel chosen explicitly:
- * path 0 = automatic (as above), 1 = tensor-core GEMM (any T; SM pairs with
- * 256x256 tiles when 2-CTA clusters can be launched), 2 = decode GEMV
- * (T <= 16, else I8_ERR_INVALID_ARG), 3 = tensor-core GEMM on single SMs
- * (128x256 tiles). */
+ * path 0 = automatic: the decode GEMV for T <= 16; for larger T the
+ * tensor-core GEMM on single SMs when the problem has fewer than 8 waves of
+ * 256x256 tiles for the SM pairs, else on SM pairs; 1 = tensor-core GEMM
+ * (any T; SM pairs with 256x256 tiles when 2-CTA clusters can be launched);
+ * 2 = decode GEMV (T <= 16, else I8_ERR_INVALID_ARG); 3 = tensor-core GEMM
+ * on single SMs (128x256 tiles). */
 i8_status int8_linear_forward_path(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
                                    const void* bias, int64_t N, float threshold, void* Y, int32_t* idx,
                                    int32_t* n_out, void* workspace, size_t workspace_bytes, int path,
@@ -340,6 +342,13 @@ i8_status int8_linear_forward_sharded(const void* X, int dtype, int64_t T, int64
                                       void* const* Y_dst, int n_dst, int64_t ldY, int64_t col_offset,
                                       int32_t* idx, int32_t* n_out, void* workspace, size_t workspace_bytes,
                                       int path, cudaStream_t stream);
+
+/* Which product kernel a forward of T x K -> N on `path` (as
+ * int8_linear_forward_path) runs on the current device: 1 = tensor-core GEMM
+ * on SM pairs, 2 = decode GEMV, 3 = tensor-core GEMM on single SMs; -1 for
+ * arguments the forward would reject or no sm_100 device.  Host-only
+ * apart from reading device attributes. */
+int int8_linear_product_kernel(int64_t T, int64_t K, int64_t N, int path);
 
 /* int8_outlier_threshold_bits for element type `dtype`: the largest magnitude
  * pattern of that type (bf16: 0..0x7f80) whose value is <= threshold.

@@ -121,9 +121,26 @@ inline i8_status cuda_status(cudaError_t e) {
 
 // The product kernel: decode GEMV, or the tensor-core GEMM on SM pairs (the
 // single-SM GEMM when pairs are not launchable or when asked for explicitly).
+// Which product kernel a forward of T x K -> N on `path` runs.  Automatic: the
+// decode GEMV for T <= 16; the single-SM GEMM for problems of fewer than 8
+// waves of 256 x 256 pair tiles (measured: the pair kernel's advantage in
+// operand traffic pays off only on long runs of tiles); the SM-pair GEMM
+// otherwise, or wherever 2-CTA clusters cannot be launched.
+int product_kernel(int64_t T, int64_t N, int path) {
+  if (path == kPathDecode || (path == kPathAuto && T <= kDecodeMaxT)) return kPathDecode;
+  if (path == kPathTensorCoreSingleSM) return kPathTensorCoreSingleSM;
+  const int pairs = pair_kernel_max_clusters();
+  if (pairs <= 0) return kPathTensorCoreSingleSM;
+  if (path == kPathAuto) {
+    const int64_t tiles = ((T + 255) / 256) * ((N + 255) / 256);
+    if (tiles < 8 * static_cast<int64_t>(pairs)) return kPathTensorCoreSingleSM;
+  }
+  return kPathTensorCore;
+}
+
 cudaError_t launch_product(const GemmArgs& a, int path, bool gemv, int num_sms, cudaStream_t stream) {
   if (gemv) return launch_gemv_decode(a, num_sms, stream);
-  if (path != kPathTensorCoreSingleSM && pair_kernel_max_clusters() > 0) return launch_gemm_tc2(a, stream);
+  if (product_kernel(a.T, a.N, path) == kPathTensorCore) return launch_gemm_tc2(a, stream);
   return launch_gemm_tc(a, num_sms, stream);
 }
 
@@ -238,6 +255,14 @@ const char* int8_status_string(int status) {
 int int8_version(void) { return 100; }
 
 uint32_t int8_outlier_threshold_bits(float threshold) { return threshold_bits(threshold, kF16); }
+
+int int8_linear_product_kernel(int64_t T, int64_t K, int64_t N, int path) {
+  if (!shape_ok(T, K, N) || path < kPathAuto || path > kPathTensorCoreSingleSM) return -1;
+  if (path == kPathDecode && T > kDecodeMaxT) return -1;
+  int num_sms = 0;
+  if (device_info(&num_sms) != I8_OK) return -1;
+  return product_kernel(T, N, path);
+}
 
 uint32_t int8_outlier_threshold_bits_ex(float threshold, int dtype) {
   if (!dtype_ok(dtype)) return 0xfffffffeu;

@@ -81,6 +81,7 @@ SIGNATURES = {
     "int8_linear_forward_sharded": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _I64, _F32,
                                            ctypes.POINTER(ctypes.c_void_p), _I32, _I64, _I64, _P, _P, _P, _SZ,
                                            _I32, _P]),
+    "int8_linear_product_kernel": (_I32, [_I64, _I64, _I64, _I32]),
     "int8_linear_forward_host_async": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _I64, _F32, _P, _P, _P, _P, _SZ,
                                               _P]),
 }
@@ -299,6 +300,12 @@ def int8_linear_forward_sharded(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Te
                                            _ptr(workspace), workspace.numel(), int(path), _stream(stream))
     _check("int8_linear_forward_sharded", st)
     return idx, n_out, workspace
+
+
+def int8_linear_product_kernel(T: int, K: int, N: int, path: int = PATH_AUTO) -> int:
+    """The product kernel a forward runs: PATH_TENSOR_CORE (SM pairs), PATH_DECODE or
+    PATH_TENSOR_CORE_1SM; -1 if the forward would reject the arguments."""
+    return int(lib().int8_linear_product_kernel(T, K, N, int(path)))
 
 
 def int8_check_status(workspace: torch.Tensor, stream=None) -> tuple[int, int]:
