@@ -111,10 +111,9 @@ i8_status int8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t*
                               cudaStream_t stream);
 
 /* As int8_linear_forward, with the product kernel chosen explicitly:
- * path 0 = automatic: the decode GEMV for T <= 16; for larger T the
- * tensor-core GEMM on single SMs when the problem has fewer than 8 waves of
- * 256x256 tiles for the SM pairs, else on SM pairs; 1 = tensor-core GEMM
- * (any T; SM pairs with 256x256 tiles when 2-CTA clusters can be launched);
+ * path 0 = automatic: the decode GEMV for T <= 16, else the tensor-core GEMM
+ * as path 1; 1 = tensor-core GEMM (any T; SM pairs with 256x512 tiles when
+ * 2-CTA clusters can be launched, else single SMs);
  * 2 = decode GEMV (T <= 16, else I8_ERR_INVALID_ARG); 3 = tensor-core GEMM
  * on single SMs (128x256 tiles). */
 i8_status int8_linear_forward_path(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,

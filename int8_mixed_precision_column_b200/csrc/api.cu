@@ -122,19 +122,15 @@ inline i8_status cuda_status(cudaError_t e) {
 // The product kernel: decode GEMV, or the tensor-core GEMM on SM pairs (the
 // single-SM GEMM when pairs are not launchable or when asked for explicitly).
 // Which product kernel a forward of T x K -> N on `path` runs.  Automatic: the
-// decode GEMV for T <= 16; the single-SM GEMM for problems of fewer than 8
-// waves of 256 x 256 pair tiles (measured: the pair kernel's advantage in
-// operand traffic pays off only on long runs of tiles); the SM-pair GEMM
-// otherwise, or wherever 2-CTA clusters cannot be launched.
+// decode GEMV for T <= 16, else the SM-pair GEMM (256 x 512 tiles; measured
+// at least as fast as the single-SM GEMM from under one wave of tiles up, to
+// within 1 %), or the single-SM GEMM wherever 2-CTA clusters cannot be
+// launched.
 int product_kernel(int64_t T, int64_t N, int path) {
+  (void)N;
   if (path == kPathDecode || (path == kPathAuto && T <= kDecodeMaxT)) return kPathDecode;
   if (path == kPathTensorCoreSingleSM) return kPathTensorCoreSingleSM;
-  const int pairs = pair_kernel_max_clusters();
-  if (pairs <= 0) return kPathTensorCoreSingleSM;
-  if (path == kPathAuto) {
-    const int64_t tiles = ((T + 255) / 256) * ((N + 255) / 256);
-    if (tiles < 8 * static_cast<int64_t>(pairs)) return kPathTensorCoreSingleSM;
-  }
+  if (pair_kernel_max_clusters() <= 0) return kPathTensorCoreSingleSM;
   return kPathTensorCore;
 }
 

@@ -3,19 +3,26 @@
 // Same computation as gemm_tc.cu (int8 product over the non-outlier columns,
 // fp16 product over the outlier columns, dequantise with the row and column
 // absmax constants and add the bias: steps 2-3 of "Core idea of LLM.int8()" on
-// the Hugging Face integration page), with the output tile of a 2-CTA cluster
-// computed by one tcgen05.mma.cta_group::2 of M=256, N=256:
-//   * CTA r of the pair holds rows [128r, 128r+128) of the A tile and rows
-//     [128r, 128r+128) of the B tile (B is split along N between the CTAs),
-//     so each SM streams 32 KB per 128-byte K-block instead of 48 KB;
-//   * each CTA's TMEM holds its 128 output rows x 256 columns;
+// the Hugging Face integration page).  A 2-CTA cluster computes a 256 x 512
+// output tile with two tcgen05.mma.cta_group::2 of M=256, N=256 per K-step:
+//   * CTA r of the pair holds rows [128r, 128r+128) of the A tile and, for
+//     each N half h, rows [256h + 128r, 256h + 128r + 128) of the B tile, so an
+//     SM streams 48 KB per 128-byte K-block for 128 x 512 outputs (a 256 x 256
+//     pair tile streams 32 KB for 128 x 256: a third more bytes per MAC, and
+//     operand traffic from L2 is what bounds the full grid);
+//   * each CTA's TMEM (512 columns) holds its 128 output rows x 512 columns,
+//     one tile at a time: the epilogue of a tile does not overlap the next
+//     tile's MMAs (measured: the traffic saving outweighs that);
 //   * the even CTA (leader) issues the MMAs; both CTAs' TMA loads complete on
 //     the leader's "full" barrier, and the leader's commits arrive on both
-//     CTAs' "empty" and "TMEM full" barriers;
-//   * both CTAs' epilogues arrive on the leader's "TMEM empty" barrier.
-// Outlier columns (the 16-bit product): a kind::f16 MMA accumulates them into a
-// second (fp32) TMEM accumulator after the int8 K-blocks; TMEM then holds one
-// tile (int32 + fp32), otherwise two int32 accumulators are double-buffered.
+//     CTAs' "empty", "TMEM full" and "outliers added" barriers;
+//   * both CTAs' epilogues arrive on the leader's "TMEM empty" and "partials
+//     written" barriers.
+// Outlier columns (the 16-bit product), with TMEM full: after the int8
+// K-blocks the epilogue rewrites each accumulator in place as the fp32 partial
+// output acc * sA * SCB / 127^2 + bias (tcgen05.st), the leader then issues
+// the kind::f16 MMAs over the outlier columns accumulating onto it, and a
+// second epilogue pass converts to the 16-bit output.
 // No TMA load uses cluster multicast: each CTA loads its own halves.
 #include <cuda.h>
 
@@ -25,23 +32,24 @@ namespace i8mp {
 namespace {
 
 constexpr int BM = 128;           // rows per CTA (256 per pair)
-constexpr int BN = 256;           // output columns per tile
-constexpr int BN_HALF = BN / 2;   // B rows loaded per CTA
+constexpr int BN = 512;           // output columns per tile
+constexpr int BN_MMA = 256;       // N of one pair MMA
+constexpr int BN_BOX = 128;       // B rows per CTA per MMA
 constexpr int BKB = 128;          // bytes of K per stage
-constexpr int STAGES = 5;
+constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BKB;       // 16 KB
-constexpr int B_BYTES = BN_HALF * BKB;  // 16 KB
+constexpr int B_BYTES = 2 * BN_BOX * BKB;  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int THREADS = 64 + NUM_EPI_WARPS * 32;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
 constexpr int GROUP_M = 8;  // pair tiles (256 rows) per raster group
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC_I8 = idesc_i8_s32(2 * BM, BN);
+constexpr uint32_t IDESC_I8 = idesc_i8_s32(2 * BM, BN_MMA);
 constexpr uint16_t PAIR_MASK = 0x3;
 
 constexpr uint32_t W_EMPTY = 0x201, W_FULL = 0x202, W_TEMPTY = 0x203, W_TFULL = 0x204, W_DRAIN = 0x205,
-                   W_TEARDOWN = 0x206;
+                   W_TEARDOWN = 0x206, W_MID = 0x207, W_OFULL = 0x208;
 
 struct Params {
   int64_t T, N, K;
@@ -74,12 +82,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     gemm_i8_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmAo, const __grid_constant__ CUtensorMap tmBo,
                        const Params p) {
-  constexpr uint32_t kIdescO = idesc_f16_f32(2 * BM, BN, Elem<TE>::kMmaFormat);  // 16-bit outlier MMA
+  constexpr uint32_t kIdescO = idesc_f16_f32(2 * BM, BN_MMA, Elem<TE>::kMmaFormat);  // 16-bit outlier MMA
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];   // used in the leader only
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t tfull_bar[2];
-  __shared__ __align__(8) uint64_t tempty_bar[2];      // used in the leader only
+  __shared__ __align__(8) uint64_t tfull_bar;         // int8 product in TMEM
+  __shared__ __align__(8) uint64_t tempty_bar;        // TMEM free again (used in the leader only)
+  __shared__ __align__(8) uint64_t mid_bar;           // fp32 partial outputs in TMEM (leader only)
+  __shared__ __align__(8) uint64_t ofull_bar;         // outlier product added
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
@@ -100,10 +110,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], 2 * NUM_EPI_WARPS);
-    }
+    mbar_init(&tfull_bar, 1);
+    mbar_init(&tempty_bar, 2 * NUM_EPI_WARPS);
+    mbar_init(&mid_bar, 2 * NUM_EPI_WARPS);
+    mbar_init(&ofull_bar, 1);
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
     fence_barrier_init();
@@ -130,8 +140,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int n_out = (p.n_out != nullptr && p.mode == 0) ? __ldcg(p.n_out) : 0;
   const int nkb_o = (n_out + 63) / 64;
   const int nkb = p.nkb_i8 + nkb_o;
-  const bool has_out = nkb_o > 0;                            // outliers on tensor cores (fp32 TMEM)
-  const int nbuf = has_out ? 1 : 2;
+  const bool has_out = nkb_o > 0;  // outlier product accumulated onto the fp32 partial outputs in TMEM
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer (both CTAs)
@@ -146,7 +155,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         int m_blk, n_blk;
         tile_coords(tile, num_m, num_n, m_blk, n_blk);
         const int row_a = m_blk * 2 * BM + static_cast<int>(rank) * BM;
-        const int row_b = n_blk * BN + static_cast<int>(rank) * BN_HALF;
+        const int row_b = n_blk * BN + static_cast<int>(rank) * BN_BOX;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty_bar[s], ph ^ 1u, &abort_sh, p.st, W_EMPTY)) {
             ok = false;
@@ -159,10 +168,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (kb < p.nkb_i8) {
             tma_load_2d_pair(sa, &tmA, fb, kb * BKB, row_a);
             tma_load_2d_pair(sb, &tmB, fb, kb * BKB, row_b);
+            tma_load_2d_pair(sb + BN_BOX * BKB, &tmB, fb, kb * BKB, row_b + BN_MMA);
           } else {
             const int ko = kb - p.nkb_i8;
             tma_load_2d_pair(sa, &tmAo, fb, ko * 64, row_a);
             tma_load_2d_pair(sb, &tmBo, fb, ko * 64, row_b);
+            tma_load_2d_pair(sb + BN_BOX * BKB, &tmBo, fb, ko * 64, row_b + BN_MMA);
           }
           ++issued[s];
           if (++s == STAGES) {
@@ -190,13 +201,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       int it = 0;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++it) {
-        const int buf = it % nbuf;
-        const uint32_t aph = static_cast<uint32_t>((it / nbuf) & 1);
-        if (!mbar_wait_cluster(&tempty_bar[buf], aph ^ 1u, &abort_sh, p.st, W_TEMPTY)) break;
+        const uint32_t aph = static_cast<uint32_t>(it & 1);
+        if (!mbar_wait_cluster(&tempty_bar, aph ^ 1u, &abort_sh, p.st, W_TEMPTY)) break;
         tc_fence_after();
-        const uint32_t d_i32 = tmem_base + static_cast<uint32_t>(buf) * 256u;
-        const uint32_t d_f32 = tmem_base + 256u;
         for (int kb = 0; kb < nkb; ++kb) {
+          if (kb == p.nkb_i8) {
+            // int8 product done; the epilogue rewrites it in place as fp32
+            // partial outputs, onto which the outlier MMAs accumulate
+            mma_commit_pair(&tfull_bar, PAIR_MASK);
+            if (!mbar_wait_cluster(&mid_bar, aph, &abort_sh, p.st, W_MID)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
           if (!mbar_wait(&full_bar[s], ph, &abort_sh, p.st, W_FULL)) {
             ok = false;
             break;
@@ -205,15 +223,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
           const uint64_t adesc = sw128_kmajor_desc(a_addr);
           const uint64_t bdesc = sw128_kmajor_desc(a_addr + A_BYTES);
+          const uint64_t bdesc2 = sw128_kmajor_desc(a_addr + A_BYTES + BN_BOX * BKB);
           if (kb < p.nkb_i8) {
             #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_i8_pair(d_i32, adesc + 2u * kk, bdesc + 2u * kk, IDESC_I8, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+              mma_i8_pair(tmem_base, adesc + 2u * kk, bdesc + 2u * kk, IDESC_I8, accum);
+              mma_i8_pair(tmem_base + 256u, adesc + 2u * kk, bdesc2 + 2u * kk, IDESC_I8, accum);
+            }
           } else {
-            const int ko = kb - p.nkb_i8;
             #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_pair(d_f32, adesc + 2u * kk, bdesc + 2u * kk, kIdescO, (ko | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              mma_f16_pair(tmem_base, adesc + 2u * kk, bdesc + 2u * kk, kIdescO, 1u);
+              mma_f16_pair(tmem_base + 256u, adesc + 2u * kk, bdesc2 + 2u * kk, kIdescO, 1u);
+            }
           }
           mma_commit_pair(&empty_bar[s], PAIR_MASK);
           if (++s == STAGES) {
@@ -221,7 +244,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             ph ^= 1u;
           }
         }
-        if (ok) mma_commit_pair(&tfull_bar[buf], PAIR_MASK);
+        if (ok) mma_commit_pair(has_out ? &ofull_bar : &tfull_bar, PAIR_MASK);
       }
       mma_commit_pair(&drain_bar, 0x1);
       volatile int never = 0;
@@ -233,98 +256,135 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int half = (warp - 2) >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     int it = 0;
+    // column scales and bias of the 32 output columns from gcol0
+    auto load_scales = [&](int64_t gcol0, float (&sc)[32], float (&bi)[32]) {
+      const bool full = gcol0 + 32 <= p.N;
+      if (full && p.vec_scb) {
+        const float4* s4 = reinterpret_cast<const float4*>(p.SCB + gcol0);
+        #pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 v = __ldg(s4 + q4);
+          sc[4 * q4] = v.x;
+          sc[4 * q4 + 1] = v.y;
+          sc[4 * q4 + 2] = v.z;
+          sc[4 * q4 + 3] = v.w;
+        }
+      } else {
+        #pragma unroll
+        for (int i = 0; i < 32; ++i) sc[i] = (gcol0 + i < p.N) ? __ldg(&p.SCB[gcol0 + i]) : 0.0f;
+      }
+      if (p.bias == nullptr) {
+        #pragma unroll
+        for (int i = 0; i < 32; ++i) bi[i] = 0.0f;
+      } else if (full && p.vec_bias) {
+        const uint4* b8 = reinterpret_cast<const uint4*>(static_cast<const TE*>(p.bias) + gcol0);
+        #pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const uint4 v = __ldg(b8 + q8);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          #pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = Elem<TE>::to_float2(w[e]);
+            bi[8 * q8 + 2 * e] = f.x;
+            bi[8 * q8 + 2 * e + 1] = f.y;
+          }
+        }
+      } else {
+        #pragma unroll
+        for (int i = 0; i < 32; ++i)
+          bi[i] = (gcol0 + i < p.N) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[gcol0 + i]) : 0.0f;
+      }
+    };
+    // 32 fp32 outputs of row `row` from gcol0 to Y (and its extra destinations)
+    auto store_y = [&](int64_t row, int64_t gcol0, const uint32_t (&packed)[16]) {
+      const int64_t off = row * p.yd.ld + gcol0;
+      TE* dst = static_cast<TE*>(p.Y) + off;
+      #pragma unroll
+      for (int g = 0; g < 4; ++g)
+        if (gcol0 + g * 8 + 8 <= p.N) {
+          const uint4 v = make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+          reinterpret_cast<uint4*>(dst)[g] = v;
+          if (p.yd.n > 0) store_extra_u4<TE>(p.yd, off + g * 8, v);
+        }
+    };
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
-      const int buf = it % nbuf;
-      const uint32_t aph = static_cast<uint32_t>((it / nbuf) & 1);
+      const uint32_t aph = static_cast<uint32_t>(it & 1);
       int m_blk, n_blk;
       tile_coords(tile, num_m, num_n, m_blk, n_blk);
       const int64_t row = static_cast<int64_t>(m_blk) * 2 * BM + static_cast<int64_t>(rank) * BM + q * 32 + lane;
       const bool row_ok = row < p.T;
-      if (!mbar_wait_cluster(&tfull_bar[buf], aph, &abort_sh, p.st, W_TFULL)) break;
+      if (!mbar_wait_cluster(&tfull_bar, aph, &abort_sh, p.st, W_TFULL)) break;
       tc_fence_after();
       const float ra = (row_ok && p.mode == 0) ? __ldg(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
-      #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        const int col0 = half * 128 + c * 32;
-        const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
-        uint32_t acc[32];
-        uint32_t fo[32];
-        tmem_ld_32x32b_x32(tmem_base + lane_base + static_cast<uint32_t>(buf) * 256u + col0, acc);
-        if (has_out) tmem_ld_32x32b_x32(tmem_base + lane_base + 256u + col0, fo);
-        tmem_ld_wait();
-        if (p.mode == 1) {
-          if (row_ok) {
-            int32_t* dst = p.acc_out + row * p.N + gcol0;
-            #pragma unroll
-            for (int g = 0; g < 8; ++g)
-              if (gcol0 + g * 4 + 4 <= p.N)
-                reinterpret_cast<int4*>(dst)[g] = make_int4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]);
-          }
-          continue;
-        }
-        float sc[32], bi[32];
-        const bool full = gcol0 + 32 <= p.N;
-        if (full && p.vec_scb) {
-          const float4* s4 = reinterpret_cast<const float4*>(p.SCB + gcol0);
-          #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 v = __ldg(s4 + q4);
-            sc[4 * q4] = v.x;
-            sc[4 * q4 + 1] = v.y;
-            sc[4 * q4 + 2] = v.z;
-            sc[4 * q4 + 3] = v.w;
-          }
-        } else {
-          #pragma unroll
-          for (int i = 0; i < 32; ++i) sc[i] = (gcol0 + i < p.N) ? __ldg(&p.SCB[gcol0 + i]) : 0.0f;
-        }
-        if (p.bias == nullptr) {
-          #pragma unroll
-          for (int i = 0; i < 32; ++i) bi[i] = 0.0f;
-        } else if (full && p.vec_bias) {
-          const uint4* b8 = reinterpret_cast<const uint4*>(static_cast<const TE*>(p.bias) + gcol0);
-          #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            const uint4 v = __ldg(b8 + q8);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = Elem<TE>::to_float2(w[e]);
-              bi[8 * q8 + 2 * e] = f.x;
-              bi[8 * q8 + 2 * e + 1] = f.y;
-            }
-          }
-        } else {
+      const uint32_t t_row = tmem_base + lane_base;
+      if (has_out) {
+        // pass 1: acc * sA * SCB / 127^2 + bias as fp32, written back in place
+        #pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          const int col0 = half * 256 + c * 32;
+          const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
+          uint32_t acc[32];
+          tmem_ld_32x32b_x32(t_row + col0, acc);
+          float sc[32], bi[32];
+          load_scales(gcol0, sc, bi);
+          tmem_ld_wait();
           #pragma unroll
           for (int i = 0; i < 32; ++i)
-            bi[i] = (gcol0 + i < p.N) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[gcol0 + i]) : 0.0f;
+            acc[i] = __float_as_uint(fmaf(static_cast<float>(static_cast<int32_t>(acc[i])), ra * sc[i], bi[i]));
+          tmem_st_32x32b_x32(t_row + col0, acc);
         }
-        uint32_t packed[16];
-        #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float y0 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i])), ra * sc[i], bi[i]);
-          float y1 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i + 1])), ra * sc[i + 1], bi[i + 1]);
-          if (has_out) {
-            y0 += __uint_as_float(fo[i]);
-            y1 += __uint_as_float(fo[i + 1]);
-          }
-          packed[i >> 1] = Elem<TE>::pack2(y0, y1);
-        }
-        if (row_ok) {
-          const int64_t off = row * p.yd.ld + gcol0;
-          TE* dst = static_cast<TE*>(p.Y) + off;
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(&mid_bar, 0);
+        if (!mbar_wait_cluster(&ofull_bar, aph, &abort_sh, p.st, W_OFULL)) break;
+        tc_fence_after();
+        // pass 2: the outlier product has been added; convert and store
+        #pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          const int col0 = half * 256 + c * 32;
+          const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
+          uint32_t yv[32];
+          tmem_ld_32x32b_x32(t_row + col0, yv);
+          tmem_ld_wait();
+          uint32_t packed[16];
           #pragma unroll
-          for (int g = 0; g < 4; ++g)
-            if (gcol0 + g * 8 + 8 <= p.N) {
-              const uint4 v = make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
-              reinterpret_cast<uint4*>(dst)[g] = v;
-              if (p.yd.n > 0) store_extra_u4<TE>(p.yd, off + g * 8, v);
+          for (int i = 0; i < 32; i += 2) packed[i >> 1] = Elem<TE>::pack2(__uint_as_float(yv[i]), __uint_as_float(yv[i + 1]));
+          if (row_ok) store_y(row, gcol0, packed);
+        }
+      } else {
+        #pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          const int col0 = half * 256 + c * 32;
+          const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
+          uint32_t acc[32];
+          tmem_ld_32x32b_x32(t_row + col0, acc);
+          tmem_ld_wait();
+          if (p.mode == 1) {
+            if (row_ok) {
+              int32_t* dst = p.acc_out + row * p.N + gcol0;
+              #pragma unroll
+              for (int g = 0; g < 8; ++g)
+                if (gcol0 + g * 4 + 4 <= p.N)
+                  reinterpret_cast<int4*>(dst)[g] = make_int4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]);
             }
+            continue;
+          }
+          float sc[32], bi[32];
+          load_scales(gcol0, sc, bi);
+          uint32_t packed[16];
+          #pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float y0 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i])), ra * sc[i], bi[i]);
+            const float y1 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i + 1])), ra * sc[i + 1], bi[i + 1]);
+            packed[i >> 1] = Elem<TE>::pack2(y0, y1);
+          }
+          if (row_ok) store_y(row, gcol0, packed);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(&tempty_bar[buf], 0);
+      if (lane == 0) mbar_arrive_cluster(&tempty_bar, 0);
     }
   }
 
@@ -405,12 +465,12 @@ cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s) {
   if (a.T == 0 || a.N == 0) return cudaSuccess;
   CUtensorMap tmA, tmB, tmAo, tmBo;
   if (!make_map(&tmA, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K, a.T, a.K, BKB, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&tmB, a.CB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K, a.N, a.K, BKB, BN_HALF)) return cudaErrorInvalidValue;
+  if (!make_map(&tmB, a.CB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K, a.N, a.K, BKB, BN_BOX)) return cudaErrorInvalidValue;
   const bool outl = a.mode == 0 && a.n_out != nullptr && a.Xo != nullptr && a.Wo != nullptr;
   const CUtensorMapDataType t16 = a.dtype == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   if (outl) {
     if (!make_map(&tmAo, a.Xo, t16, a.ldo, a.T, a.ldo * 2, 64, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&tmBo, a.Wo, t16, a.ldo, a.N, a.ldo * 2, 64, BN_HALF))
+    if (!make_map(&tmBo, a.Wo, t16, a.ldo, a.N, a.ldo * 2, 64, BN_BOX))
       return cudaErrorInvalidValue;
   } else {
     tmAo = tmA;

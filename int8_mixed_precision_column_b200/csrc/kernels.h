@@ -106,8 +106,8 @@ inline YDst make_ydst(const GemmArgs& a) {
 // kind::f16 outlier product and dequant/bias epilogue.
 cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t s);
 
-// Prefill, pair-of-SMs version: 2-CTA clusters, tcgen05.mma.cta_group::2 with
-// 256 x 256 tiles.  Returns cudaErrorNotSupported if such clusters cannot be
+// Prefill, pair-of-SMs version: 2-CTA clusters, two tcgen05.mma.cta_group::2
+// of 256 x 256 per K-step for a 256 x 512 tile.  Returns cudaErrorNotSupported if such clusters cannot be
 // launched on the current device.
 cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s);
 int pair_kernel_max_clusters();
