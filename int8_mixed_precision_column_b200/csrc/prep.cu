@@ -266,8 +266,12 @@ __device__ __forceinline__ uint32_t chunk_max_mag_kept(const uint4& v, uint32_t 
 // For |y| < 0.5 the code is 0 (tested explicitly: just below 0.5, |y| + 0.5
 // rounds up to 1.0 in fp32).  |y| <= 127 * (1 + 2^-24)^2 < 127.5 keeps the
 // result within +-127 without a clamp.
+// Round half away from zero for |y| <= 127.5 (the codes' range): with
+// n = floor(|y| + 0.5), an integer and so exactly representable, the fp32 sum
+// |y| + 0.5 rounded toward zero lies in [n, n + 1), and truncating it gives n.
+// (Rounded to nearest, the sum fails below 0.5: 0.49999997 + 0.5 -> 1.0.)
 __device__ __forceinline__ int round_away_code(float y) {
-  return (fabsf(y) < 0.5f) ? 0 : __float2int_rz(y + copysignf(0.5f, y));
+  return __float2int_rz(copysignf(__fadd_rz(fabsf(y), 0.5f), y));
 }
 
 template <typename TE>

@@ -82,6 +82,27 @@ def test_bf16_forward_matches_oracle(path, T, K, N, planted, thr):
     assert err <= O.y_tolerance_bf16(r["Y"]), err
 
 
+def test_bf16_pair_tiles_outnumber_pairs():
+    """bf16 through the SM-pair kernel with 85 output tiles for 74 pairs, two
+    outlier K-blocks and ragged last tiles; sampled rows, every column."""
+    T, K, N = 1100, 336, 8208
+    X, W, b = _bf16_problem(T, K, N, 70, 6.0, seed=5)
+    CB, SCB = native.int8_quantize_weight(W.cuda())
+    Y, idx, n_out, ws = native.int8_linear_forward(X.cuda(), CB, SCB, b.cuda(), 6.0, path=native.PATH_TENSOR_CORE)
+    st, where = native.int8_check_status(ws)
+    assert st == 0, f"device status {st} at {where:#x} ({native.int8_last_cuda_error()})"
+    rows = list(range(0, T, 37)) + [T - 1]
+    r = O.linear_forward_bf16(_u16(X), CB.cpu().numpy(), SCB.cpu().numpy(), _u16(b), 6.0, rows=rows)
+    n = int(n_out.item())
+    assert n == r["n_out"] > 64 and np.array_equal(idx[:n].cpu().numpy(), r["idx"])
+    v = native.workspace_views(ws, T, K, N, torch.bfloat16)
+    rt = torch.as_tensor(rows, device="cuda")
+    assert np.array_equal(v["Xq"][rt].cpu().numpy(), r["Xq"])
+    assert np.array_equal(v["sA"][rt].cpu().numpy(), r["sA"])
+    err = np.abs(Y[rt].float().cpu().numpy().astype(np.float64) - r["Y"]).max()
+    assert err <= O.y_tolerance_bf16(r["Y"]), err
+
+
 def test_bf16_no_bias_and_every_column_flagged():
     T, K, N = 24, 128, 64
     X, W, _ = _bf16_problem(T, K, N, 0, 0.0, seed=11, bias=False)

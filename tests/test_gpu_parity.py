@@ -140,6 +140,19 @@ def test_ragged_tensor_core(T, K, N, planted, thr, path):
     check_forward(p, gpu_forward(p, path))
 
 
+@pytest.mark.parametrize("T,N", [(1100, 8208), (513, 38416)])
+def test_pair_tiles_outnumber_pairs(T, N):
+    """More 256 x 512 output tiles than SM pairs, so pairs take several in turn
+    (TMEM and the per-tile barriers reused with the outlier product added in
+    place), two outlier K-blocks, and a ragged last tile in both directions
+    (T = 1100: 76 rows; T = 513: one row; N: 16 columns), whose output the TMA
+    stores clip.  Sampled rows against the oracle, every column."""
+    p = workloads.make_problem("multi", T, 336, N, n_planted=70, bias_std=0.01, seed=T + N)
+    g = gpu_forward(p, "tc")
+    assert g["n_out"] > 64
+    check_forward(p, g, rows=list(range(0, T, 37)) + [T - 1])
+
+
 @pytest.mark.parametrize("T,K,N,planted,path", [
     (300, 20480, 256, 9, "tc"),       # K > 16384, few rows: two-pass CTA-per-row quantisation
     (2048, 20480, 128, 9, "tc"),      # K > 16384, many rows: warp-per-row quantisation
