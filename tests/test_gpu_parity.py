@@ -226,6 +226,22 @@ def test_exact_threshold_value_not_flagged():
     check_forward(p, g, check_wo=False)
 
 
+@pytest.mark.parametrize("T,K,N,path,expect", [
+    (1, 14336, 57344, "auto", "decode"), (16, 4096, 4096, "auto", "decode"),
+    (17, 4096, 4096, "auto", "tc"), (2048, 4096, 4096, "auto", "tc"), (8192, 14336, 57344, "auto", "tc"),
+    (4, 4096, 4096, "tc", "tc"), (2048, 4096, 4096, "tc1", "tc1"), (16, 4096, 4096, "decode", "decode"),
+])
+def test_product_kernel_choice(T, K, N, path, expect):
+    """The automatic path: the decode GEMV for T <= 16, the SM-pair GEMM above
+    (2-CTA clusters launch on B200); explicit paths are honoured."""
+    assert native.int8_linear_product_kernel(T, K, N, PATHS[path]) == PATHS[expect]
+
+
+def test_product_kernel_choice_rejects_bad_arguments():
+    assert native.int8_linear_product_kernel(17, 4096, 4096, native.PATH_DECODE) == -1
+    assert native.int8_linear_product_kernel(4, 4100, 4096, native.PATH_AUTO) == -1
+
+
 def test_empty_batch():
     p = workloads.make_problem("empty", 0, 64, 64, seed=7)
     CB, SCB = native.int8_quantize_weight(p.W.cuda())
