@@ -319,7 +319,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         uint4* d = reinterpret_cast<uint4*>(buf + lane * 64);
         #pragma unroll
-        for (int g = 0; g < 4; ++g) d[g] = make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+        for (int g = 0; g < 4; ++g)
+          d[g] = make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -383,7 +384,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld_wait();
           uint32_t packed[16];
           #pragma unroll
-          for (int i = 0; i < 32; i += 2) packed[i >> 1] = Elem<TE>::pack2(__uint_as_float(yv[i]), __uint_as_float(yv[i + 1]));
+          for (int i = 0; i < 32; i += 2)
+            packed[i >> 1] = Elem<TE>::pack2(__uint_as_float(yv[i]), __uint_as_float(yv[i + 1]));
           store_y(row, row_ok, row - lane, gcol0, packed);
         }
       } else {
@@ -400,7 +402,8 @@ __global__ void __launch_bounds__(THREADS, 1)
               #pragma unroll
               for (int g = 0; g < 8; ++g)
                 if (gcol0 + g * 4 + 4 <= p.N)
-                  reinterpret_cast<int4*>(dst)[g] = make_int4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]);
+                  reinterpret_cast<int4*>(dst)[g] =
+                      make_int4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]);
             }
             continue;
           }

@@ -107,8 +107,9 @@ inline YDst make_ydst(const GemmArgs& a) {
 cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t s);
 
 // Prefill, pair-of-SMs version: 2-CTA clusters, two tcgen05.mma.cta_group::2
-// of 256 x 256 per K-step for a 256 x 512 tile.  Returns cudaErrorNotSupported if such clusters cannot be
-// launched on the current device.
+// of 256 x 256 per K-step for a 256 x 512 tile.  Returns
+// cudaErrorNotSupported if such clusters cannot be launched on the current
+// device.
 cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s);
 int pair_kernel_max_clusters();
 
