@@ -222,11 +222,36 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
   }
 }
 
+// Prefer L1 to shared memory: 28 % of the unified storage (the 64 KB
+// configuration) still holds the 2 CTAs per SM, and the token codes, re-read
+// from L1 by every pass, then stay there more often.  Measured at BLOOM FFN-up
+// width: 1.2 % faster at T = 1, 2.3 % at T = 16; the largest shared-memory
+// configuration doubled the time.  A hint, set once per device; a failure is
+// cleared and ignored.
+bool g_carveout_set[64] = {false};
+
+void prefer_l1(int dev) {
+  if (dev < 0 || dev >= 64 || g_carveout_set[dev]) return;
+  const int pct = 28;
+  bool ok = cudaFuncSetAttribute(gemv_i8_decode_kernel<__half, false>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout, pct) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(gemv_i8_decode_kernel<__half, true>,
+                                  cudaFuncAttributePreferredSharedMemoryCarveout, pct) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(gemv_i8_decode_kernel<__nv_bfloat16, false>,
+                                  cudaFuncAttributePreferredSharedMemoryCarveout, pct) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(gemv_i8_decode_kernel<__nv_bfloat16, true>,
+                                  cudaFuncAttributePreferredSharedMemoryCarveout, pct) == cudaSuccess;
+  if (!ok) (void)cudaGetLastError();
+  g_carveout_set[dev] = true;
+}
+
 }  // namespace
 
 cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s) {
   if (a.T == 0 || a.N == 0) return cudaSuccess;
   if (a.T > kDecodeMaxT) return cudaErrorInvalidValue;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) prefer_l1(dev);
   DvParams p;
   p.Xq = a.Xq;
   p.sA = a.sA;
