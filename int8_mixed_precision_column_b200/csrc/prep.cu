@@ -544,11 +544,28 @@ __global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
 constexpr int kSmallMaxK = 131072;
 constexpr int kSmallThreads = 512;
 constexpr int kSmallUnroll = 4;
+constexpr int64_t kSmallResidentK = static_cast<int64_t>(kSmallThreads) * kSmallUnroll * 8;
+
+// 32-bit load from the shared memory of CTA `rank` of this cluster, at the
+// offset `local` has in this CTA.
+__device__ __forceinline__ uint32_t ld_dsmem_u32(const uint32_t* local, uint32_t rank) {
+  uint32_t v;
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %1, %2;\n\tld.shared::cluster.u32 %0, [ra];\n\t}"
+      : "=r"(v)
+      : "r"(smem_u32(local)), "r"(rank)
+      : "memory");
+  return v;
+}
 
 // kResident (K <= 512 x 4 x 8): each thread keeps its 4 chunks of the CTA's own
 // row in registers from the first load to the codes; other rows are read for
 // the mask only.
-template <typename TE, bool kResident>
+// kCluster (with kResident; the T CTAs form one thread-block cluster): each
+// CTA flags only its own row, into its own shared memory, and the column mask
+// is the OR of the T CTAs' flags read through distributed shared memory,
+// instead of every CTA testing all T rows.
+template <typename TE, bool kResident, bool kCluster>
 __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
     const TE* __restrict__ X, int64_t T, int64_t K, uint32_t hbits, uint32_t* __restrict__ mask,
     uint32_t* __restrict__ prefix, int32_t* __restrict__ idx, int32_t* __restrict__ n_out_p, int8_t* __restrict__ Xq,
@@ -558,6 +575,8 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
   __shared__ uint32_t s_prefix[kSmallMaxK / 32];
   __shared__ int s_scan[kSmallThreads];
   __shared__ uint32_t s_max[kSmallThreads / 32];
+  __shared__ uint32_t s_own[kCluster ? kSmallResidentK / 32 : 1];  // this row's flags
+  static_assert(!kCluster || kResident, "the cluster form keeps the row in registers");
   griddep_launch_dependents();  // the product kernel may start its prologue
   const int64_t nv = K / 8;
   const int64_t nw = (K + 31) / 32;
@@ -573,6 +592,26 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
       v[u] = (c < nv) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
     }
   }
+  if constexpr (kCluster) {
+    for (int64_t w = threadIdx.x; w < nw; w += kSmallThreads) s_own[w] = 0;
+    __syncthreads();
+    if (on) {
+      #pragma unroll
+      for (int u = 0; u < kSmallUnroll; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(kSmallThreads) * u;
+        if (c >= nv) continue;
+        const uint32_t bits = flag_bits8<TE>(v[u], h2);
+        if (bits) atomicOr(&s_own[c >> 2], bits << ((c & 3) * 8));
+      }
+    }
+    cluster_sync();  // every CTA's flags are complete (release / acquire, cluster scope)
+    for (int64_t w = threadIdx.x; w < nw; w += kSmallThreads) {
+      uint32_t m = 0;
+      for (int64_t r = 0; r < T; ++r) m |= ld_dsmem_u32(&s_own[w], static_cast<uint32_t>(r));
+      s_mask[w] = m;
+    }
+    cluster_sync();  // no CTA reads another's flags after this; s_mask is complete
+  } else {
   for (int64_t w = threadIdx.x; w < nw; w += kSmallThreads) s_mask[w] = 0;
   __syncthreads();
   // mask: column chunk c is flagged from all T rows
@@ -609,6 +648,7 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
     }
   }
   __syncthreads();
+  }
   // prefix counts: thread i owns a contiguous run of mask words
   const int64_t per = (nw + kSmallThreads - 1) / kSmallThreads;
   const int64_t w0 = threadIdx.x * per;
@@ -701,22 +741,73 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
   for (int64_t o = n_out + threadIdx.x; o < npad; o += kSmallThreads) xo_row[o] = E::from_float(0.0f);
 }
 
+// Whether the T CTAs of the cluster form can be co-scheduled as one cluster
+// (per device, element type and T; 1 yes, -1 no, 0 not yet asked).  Clusters
+// of more than 8 CTAs need the non-portable size opt-in.
+int8_t g_cluster_ok[64][2][kDecodeMaxT + 1];
+
+template <typename TE>
+bool cluster_form_ok(int64_t T, int et) {
+  int dev = 0;
+  if (T < 2 || T > kDecodeMaxT || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  int8_t& c = g_cluster_ok[dev][et][T];
+  if (c != 0) return c > 0;
+  auto* k = prep_small_kernel<TE, true, true>;
+  bool ok = T <= 8 || cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  int n = 0;
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(T);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(T), 1, 1);
+    cfg.blockDim = dim3(kSmallThreads, 1, 1);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ok = cudaOccupancyMaxActiveClusters(&n, k, &cfg) == cudaSuccess && n > 0;
+  }
+  if (!ok) (void)cudaGetLastError();  // a refused opt-in or query only means: no cluster form
+  c = ok ? 1 : -1;
+  return ok;
+}
+
+template <typename TE>
+cudaError_t launch_prep_small_t(const TE* X, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
+                                uint32_t* prefix, int32_t* idx, int32_t* n_out, int8_t* Xq, float* sA, TE* Xo,
+                                int64_t ldo, DevStatus* st, int et, cudaStream_t s) {
+  const bool resident = K <= kSmallResidentK;
+  if (resident && cluster_form_ok<TE>(T, et)) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(T);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(T), 1, 1);
+    cfg.blockDim = dim3(kSmallThreads, 1, 1);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prep_small_kernel<TE, true, true>, X, T, K, hbits, mask, prefix, idx, n_out, Xq,
+                              sA, Xo, ldo, st);
+  }
+  auto* k = resident ? prep_small_kernel<TE, true, false> : prep_small_kernel<TE, false, false>;
+  k<<<dim3(static_cast<unsigned>(T)), kSmallThreads, 0, s>>>(X, T, K, hbits, mask, prefix, idx, n_out, Xq, sA, Xo,
+                                                              ldo, st);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_prep_small(const void* X, int dtype, int64_t T, int64_t K, uint32_t hbits, uint32_t* mask,
                               uint32_t* prefix, int32_t* idx, int32_t* n_out, int8_t* Xq, float* sA, void* Xo,
                               int64_t ldo, DevStatus* st, cudaStream_t s) {
   if (T < 1 || T > kDecodeMaxT || K > kSmallMaxK) return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>(T));
-  const bool resident = K <= static_cast<int64_t>(kSmallThreads) * kSmallUnroll * 8;
-  if (dtype == kBF16) {
-    auto* k = resident ? prep_small_kernel<__nv_bfloat16, true> : prep_small_kernel<__nv_bfloat16, false>;
-    k<<<grid, kSmallThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(X), T, K, hbits, mask, prefix, idx, n_out,
-                                      Xq, sA, static_cast<__nv_bfloat16*>(Xo), ldo, st);
-  } else {
-    auto* k = resident ? prep_small_kernel<__half, true> : prep_small_kernel<__half, false>;
-    k<<<grid, kSmallThreads, 0, s>>>(static_cast<const __half*>(X), T, K, hbits, mask, prefix, idx, n_out, Xq, sA,
-                                      static_cast<__half*>(Xo), ldo, st);
-  }
-  return cudaGetLastError();
+  if (dtype == kBF16)
+    return launch_prep_small_t(static_cast<const __nv_bfloat16*>(X), T, K, hbits, mask, prefix, idx, n_out, Xq, sA,
+                               static_cast<__nv_bfloat16*>(Xo), ldo, st, 1, s);
+  return launch_prep_small_t(static_cast<const __half*>(X), T, K, hbits, mask, prefix, idx, n_out, Xq, sA,
+                             static_cast<__half*>(Xo), ldo, st, 0, s);
 }
 
 template <typename TE>
