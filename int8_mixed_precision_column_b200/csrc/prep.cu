@@ -82,6 +82,36 @@ cudaError_t launch_quantize_weight(const void* W, int dtype, int64_t N, int64_t 
 // prefix[w] + popc(lower bits of word w).
 // ---------------------------------------------------------------------------
 constexpr int kMaskThreads = 256;
+
+// Exclusive prefix sum of v over the NT threads of the CTA (all of them call
+// it, once), by warp shuffles: inclusive scans within each warp, then one warp
+// scans the warp totals.  *total receives the sum.  s_warp holds NT/32 ints.
+template <int NT>
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total) {
+  static_assert(NT % 32 == 0 && NT / 32 <= 32, "one warp scans the warp totals");
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  int x = v;
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int t = (lane < NT / 32) ? s_warp[lane] : 0;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < NT / 32) s_warp[lane] = t;
+  }
+  __syncthreads();
+  *total = s_warp[NT / 32 - 1];
+  return (w > 0 ? s_warp[w - 1] : 0) + x - v;
+}
 constexpr int kMaskUnroll = 4;
 
 // Largest magnitude bit pattern among the 8 elements of v (16-bit max of |x|;
@@ -118,7 +148,7 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const TE* __
                                                                     uint32_t* __restrict__ prefix, int32_t* __restrict__ idx,
                                                                     int32_t* __restrict__ n_out, DevStatus* st) {
   __shared__ int s_last;
-  __shared__ int s_scan[kMaskThreads];
+  __shared__ int s_scan[kMaskThreads / 32];
   griddep_launch_dependents();  // the row quantisation may start meanwhile
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -169,15 +199,8 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const TE* __
   const int64_t w1 = min(nwords, w0 + per);
   int cnt = 0;
   for (int64_t w = w0; w < w1; ++w) cnt += __popc(__ldcg(&mask[w]));
-  s_scan[threadIdx.x] = cnt;
-  __syncthreads();
-  for (int off = 1; off < kMaskThreads; off <<= 1) {
-    int v = (threadIdx.x >= off) ? s_scan[threadIdx.x - off] : 0;
-    __syncthreads();
-    s_scan[threadIdx.x] += v;
-    __syncthreads();
-  }
-  int pos = s_scan[threadIdx.x] - cnt;
+  int total = 0;
+  int pos = block_exclusive_scan<kMaskThreads>(cnt, s_scan, &total);
   for (int64_t w = w0; w < w1; ++w) {
     uint32_t m = __ldcg(&mask[w]);
     prefix[w] = static_cast<uint32_t>(pos);
@@ -188,7 +211,7 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const TE* __
     }
   }
   if (threadIdx.x == kMaskThreads - 1) {
-    *n_out = s_scan[kMaskThreads - 1];
+    *n_out = total;
     st->counter = 0;
   }
 }
@@ -573,7 +596,7 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
   using E = Elem<TE>;
   __shared__ uint32_t s_mask[kSmallMaxK / 32];
   __shared__ uint32_t s_prefix[kSmallMaxK / 32];
-  __shared__ int s_scan[kSmallThreads];
+  __shared__ int s_scan[kSmallThreads / 32];
   __shared__ uint32_t s_max[kSmallThreads / 32];
   __shared__ uint32_t s_own[kCluster ? kSmallResidentK / 32 : 1];  // this row's flags
   static_assert(!kCluster || kResident, "the cluster form keeps the row in registers");
@@ -655,16 +678,8 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
   const int64_t w1 = min(nw, w0 + per);
   int cnt = 0;
   for (int64_t w = w0; w < w1; ++w) cnt += __popc(s_mask[w]);
-  s_scan[threadIdx.x] = cnt;
-  __syncthreads();
-  for (int off = 1; off < kSmallThreads; off <<= 1) {
-    const int v = (static_cast<int>(threadIdx.x) >= off) ? s_scan[threadIdx.x - off] : 0;
-    __syncthreads();
-    s_scan[threadIdx.x] += v;
-    __syncthreads();
-  }
-  const int n_out = s_scan[kSmallThreads - 1];
-  int pos = s_scan[threadIdx.x] - cnt;
+  int n_out = 0;
+  int pos = block_exclusive_scan<kSmallThreads>(cnt, s_scan, &n_out);
   for (int64_t w = w0; w < w1; ++w) {
     s_prefix[w] = static_cast<uint32_t>(pos);
     if (blockIdx.x == 0) {
