@@ -758,7 +758,8 @@ __global__ void __launch_bounds__(kSmallThreads) prep_small_kernel(
 
 // Whether the T CTAs of the cluster form can be co-scheduled as one cluster
 // (per device, element type and T; 1 yes, -1 no, 0 not yet asked).  Clusters
-// of more than 8 CTAs need the non-portable size opt-in.
+// of more than 8 CTAs need the non-portable size opt-in.  Written without a
+// lock: concurrent first calls ask the same question and store the same answer.
 int8_t g_cluster_ok[64][2][kDecodeMaxT + 1];
 
 template <typename TE>
