@@ -24,6 +24,9 @@
  *   - Pointers documented as "device" must be CUDA device memory of the
  *     current device; the caller owns every buffer.  The library allocates
  *     nothing and keeps no per-call state outside the caller's workspace.
+ *     Per device and process it caches device properties and what the first
+ *     launch of a kernel learns (whether its 2-CTA or T-CTA clusters can be
+ *     scheduled; a shared-memory carveout hint set on the kernel).
  *   - Calls are asynchronous on `stream` unless stated otherwise.  Argument
  *     errors are reported synchronously before any work is enqueued; launch
  *     failures are reported as I8_ERR_CUDA.  A device-side wait that gives up
