@@ -115,6 +115,22 @@ def test_small_workspace_rejected(lib):
     assert st == 2  # I8_ERR_WORKSPACE
 
 
+@pytest.mark.parametrize("which,offset", [("X", 8), ("CB", 8), ("Y", 8), ("SCB", 2), ("idx", 2), ("n_out", 2),
+                                          ("bias", 1), ("ws", 128)])
+def test_misaligned_pointers_rejected_before_any_cuda_call(lib, which, offset):
+    # X, CB and Y need 16-byte alignment (16-byte vector and TMA accesses), SCB,
+    # idx and n_out 4, the bias 2, the workspace 256 (its carve-outs); the
+    # addresses are never dereferenced: validation fails first
+    T, K, N = 4, 64, 64
+    ws_bytes = native.int8_linear_workspace_bytes(T, K, N)
+    ptr = {k: 1 << 20 for k in ("X", "CB", "SCB", "bias", "Y", "idx", "n_out", "ws")}
+    ptr[which] += offset
+    v = {k: ctypes.c_void_p(a) for k, a in ptr.items()}
+    st = lib.int8_linear_forward(v["X"], T, K, v["CB"], v["SCB"], v["bias"], N, 6.0, v["Y"], v["idx"], v["n_out"],
+                                 v["ws"], ws_bytes, None)
+    assert st == (2 if which == "ws" else 1)  # I8_ERR_WORKSPACE / I8_ERR_INVALID_ARG
+
+
 def _bf16_values():
     bits = np.arange(0, 0x10000, dtype=np.uint32)
     return bits, (bits << 16).view(np.float32)
