@@ -378,9 +378,15 @@ uint32_t int8_outlier_threshold_bits_ex(float threshold, int dtype);
  *     needs more than 4 MiB (for T = 16: K above about 87000) is rejected
  *     with I8_ERR_WORKSPACE before any work is enqueued.  T outside
  *     [1, 16] is I8_ERR_INVALID_ARG.
- *   - The first call on each device resolves the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - The first call on each device does all of this call's per-device
+ *     set-up, with that device current: it resolves the array's device
+ *     address (cudaGetSymbolAddress) and, for every T in 1..16, asks whether
+ *     the decode prep kernel's T-CTA cluster can be scheduled, and sets the
+ *     decode GEMV's shared-memory carveout hint.  One first call with any T
+ *     is enough; make it before any stream capture.  Later calls make no CUDA
+ *     call other than cudaGetDevice, the two kernel launches and the launch
+ *     error query.  A failing CUDA call is reported as I8_ERR_CUDA and its
+ *     text by int8_last_cuda_error().
  *   - Every call on a device shares the one array, and the array keeps the
  *     previous call's contents (each call clears what must start at zero).
  *     Calls that can overlap on the GPU (other streams, other host threads)

@@ -22,15 +22,26 @@ struct DevInfo {
 };
 DevInfo g_dev[kMaxDevices];
 
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// Maps a CUDA result to a status, remembering the error for int8_last_cuda_error().
+inline i8_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return I8_OK;
+  g_last_cuda_error = e;
+  return I8_ERR_CUDA;
+}
+
 i8_status device_info(int* num_sms) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return I8_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
   if (dev < 0 || dev >= kMaxDevices) return I8_ERR_UNSUPPORTED;
   DevInfo& d = g_dev[dev];
   if (!d.probed) {
     int major = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return I8_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return I8_ERR_CUDA;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_status(e);
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return cuda_status(e);
     d.sm100 = (major == 10);
     d.num_sms = sms;
     d.probed = true;
@@ -110,14 +121,6 @@ uint32_t threshold_bits(float thr, int dtype = kF16) {
 
 inline bool dtype_ok(int dtype) { return dtype == kF16 || dtype == kBF16; }
 
-thread_local cudaError_t g_last_cuda_error = cudaSuccess;
-
-// Maps a CUDA result to a status, remembering the error for int8_last_cuda_error().
-inline i8_status cuda_status(cudaError_t e) {
-  if (e == cudaSuccess) return I8_OK;
-  g_last_cuda_error = e;
-  return I8_ERR_CUDA;
-}
 
 // The product kernel: decode GEMV, or the tensor-core GEMM on SM pairs (the
 // single-SM GEMM when pairs are not launchable or when asked for explicitly).
@@ -161,7 +164,7 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   if (st != I8_OK) return st;
 
   auto mark = [&](int i) -> bool {
-    return events == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) == cudaSuccess;
+    return events == nullptr || cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream)) == I8_OK;
   };
   if (!mark(0)) return I8_ERR_CUDA;
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -171,10 +174,11 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   // in shared memory; otherwise status word + mask start at zero
   const bool small_prep = gemv && T >= 1;
   cudaError_t e = small_prep ? cudaSuccess : cudaMemsetAsync(w, 0, L.mask + mask_bytes, stream);
-  if (e != cudaSuccess) return I8_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
   if (T == 0) {
     e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
-    return (e == cudaSuccess && mark(1) && mark(2) && mark(3)) ? I8_OK : I8_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
+    return (mark(1) && mark(2) && mark(3)) ? I8_OK : I8_ERR_CUDA;
   }
 
   DevStatus* dst = reinterpret_cast<DevStatus*>(w + L.status);
@@ -189,18 +193,21 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   if (small_prep) {
     // one kernel for the outlier pass and the row quantisation
     e = launch_prep_small(X, dtype, T, K, hb, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, dst, stream);
-    if (e != cudaSuccess || !mark(1) || !mark(2)) return I8_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
+    if (!mark(1) || !mark(2)) return I8_ERR_CUDA;
   } else {
     if (hb == 0xffffffffu)
       e = cudaMemsetAsync(n_out, 0, sizeof(int32_t), stream);
     else
       e = launch_outliers(X, dtype, T, K, hb, mask, prefix, idx, n_out, dst, stream);
-    if (e != cudaSuccess || !mark(1)) return I8_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
+    if (!mark(1)) return I8_ERR_CUDA;
     // programmatic launches only directly after one of our kernels
     const bool after_outliers = (hb != 0xffffffffu);
     e = launch_rowquant(X, dtype, T, K, mask, prefix, idx, n_out, Xq, sA, Xo, L.ldo, CB, SCB, N, Wo, !gemv, Wf,
                         num_sms, dst, after_outliers, stream);
-    if (e != cudaSuccess || !mark(2)) return I8_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
+    if (!mark(2)) return I8_ERR_CUDA;
   }
 
   GemmArgs a;
@@ -228,11 +235,18 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   a.n_ydst = n_ydst;
   for (int d = 0; d < n_ydst; ++d) a.ydst[d] = ydst[d];
   e = launch_product(a, path, gemv, num_sms, stream);
-  if (e != cudaSuccess || !mark(3)) return I8_ERR_CUDA;
-  return I8_OK;
+  if (e != cudaSuccess) return cuda_status(e);
+  return mark(3) ? I8_OK : I8_ERR_CUDA;
 }
 
 }  // namespace
+
+namespace i8mp {
+cudaError_t note_cuda_error(cudaError_t e) {
+  if (e != cudaSuccess) g_last_cuda_error = e;
+  return e;
+}
+}  // namespace i8mp
 
 extern "C" {
 
@@ -388,7 +402,8 @@ i8_status int8_linear_forward_fp16w_ex(const void* X, int dtype, int64_t T, int6
   i8_status st = device_info(&num_sms);
   if (st != I8_OK) return st;
   // the weight is quantised anew in every forward (Linear8bitLt, has_fp16_weights=True)
-  if (launch_quantize_weight(W, dtype, N, K, CB, SCB, stream) != cudaSuccess) return I8_ERR_CUDA;
+  const cudaError_t e = launch_quantize_weight(W, dtype, N, K, CB, SCB, stream);
+  if (e != cudaSuccess) return cuda_status(e);
   return forward_impl(X, T, K, CB, SCB, bias, N, threshold, Y, idx, n_out, workspace, L.total, 0, nullptr, stream,
                       dtype, W);
 }
@@ -422,17 +437,17 @@ static i8_status host_forward(const void* X_host, int dtype, int64_t T, int64_t 
   int32_t* nd = reinterpret_cast<int32_t*>(w + H.n_out);
   const size_t xbytes = static_cast<size_t>(T) * K * 2;
   const size_t ybytes = static_cast<size_t>(T) * N * 2;
-  if (xbytes && cudaMemcpyAsync(Xd, X_host, xbytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+  if (xbytes && cuda_status(cudaMemcpyAsync(Xd, X_host, xbytes, cudaMemcpyHostToDevice, stream)) != I8_OK)
     return I8_ERR_CUDA;
   i8_status st = forward_impl(Xd, T, K, CB, SCB, bias, N, threshold, Yd, idxd, nd, workspace, L.total, 0, nullptr,
                               stream, dtype);
   if (st != I8_OK) return st;
-  if (ybytes && cudaMemcpyAsync(Y_host, Yd, ybytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+  if (ybytes && cuda_status(cudaMemcpyAsync(Y_host, Yd, ybytes, cudaMemcpyDeviceToHost, stream)) != I8_OK)
     return I8_ERR_CUDA;
-  if (idx_host && cudaMemcpyAsync(idx_host, idxd, static_cast<size_t>(K) * 4, cudaMemcpyDeviceToHost, stream) !=
-                      cudaSuccess)
+  if (idx_host && cuda_status(cudaMemcpyAsync(idx_host, idxd, static_cast<size_t>(K) * 4, cudaMemcpyDeviceToHost,
+                                              stream)) != I8_OK)
     return I8_ERR_CUDA;
-  if (n_out_host && cudaMemcpyAsync(n_out_host, nd, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+  if (n_out_host && cuda_status(cudaMemcpyAsync(n_out_host, nd, 4, cudaMemcpyDeviceToHost, stream)) != I8_OK)
     return I8_ERR_CUDA;
   return sync ? int8_check_status(workspace, nullptr, stream) : I8_OK;
 }
@@ -463,7 +478,7 @@ i8_status int8_gemm_i32(const int8_t* Xq, int64_t T, int64_t K, const int8_t* CB
   int num_sms = 0;
   i8_status st = device_info(&num_sms);
   if (st != I8_OK) return st;
-  if (cudaMemsetAsync(workspace, 0, sizeof(DevStatus), stream) != cudaSuccess) return I8_ERR_CUDA;
+  if (cuda_status(cudaMemsetAsync(workspace, 0, sizeof(DevStatus), stream)) != I8_OK) return I8_ERR_CUDA;
   if (T == 0) return I8_OK;
   GemmArgs a;
   std::memset(&a, 0, sizeof(a));

@@ -42,6 +42,7 @@ struct Elem<__half> {
   __device__ static __forceinline__ float mag_to_float(uint32_t bits) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
   }
+  __device__ static __forceinline__ __half from_bits(uint16_t b) { return __ushort_as_half(b); }
 };
 
 template <>
@@ -64,6 +65,7 @@ struct Elem<__nv_bfloat16> {
     return *reinterpret_cast<uint32_t*>(&m);
   }
   __device__ static __forceinline__ float mag_to_float(uint32_t bits) { return __uint_as_float(bits << 16); }
+  __device__ static __forceinline__ __nv_bfloat16 from_bits(uint16_t b) { return __ushort_as_bfloat16(b); }
 };
 
 // ---------------------------------------------------------------------------
@@ -199,6 +201,24 @@ __device__ __forceinline__ void bulk_wait() {
 __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int32_t x, int32_t y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
                ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+// L2 eviction-priority policies for the cache-hinted bulk copies.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// tma_store_2d with an L2 eviction policy for the written lines.
+__device__ __forceinline__ void tma_store_2d_hint(const void* tmap, const void* smem_src, int32_t x, int32_t y,
+                                                  uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;"
+               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(smem_src)), "r"(x), "r"(y), "l"(policy)
                : "memory");
 }
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy.
@@ -388,6 +408,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const void* tma
       : "memory");
 }
 
+// tma_load_2d_pair with an L2 eviction policy for the loaded lines.
+__device__ __forceinline__ void tma_load_2d_pair_hint(void* smem_dst, const void* tmap, uint32_t bar_cluster_addr,
+                                                      int32_t x, int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster_addr), "r"(x), "r"(y),
+        "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_dst, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_dst)),
                "r"(ncols)
@@ -446,6 +477,58 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Reads of what the preceding kernel wrote, in a kernel launched with
+// programmatic stream serialisation.  Such a kernel starts while its
+// predecessor still runs, so every one of these reads
+//  * must stay behind griddep_wait().  The wait is an opaque asm statement to
+//    the compiler.  A plain load through a `const T* __restrict__` kernel
+//    argument is, for the compiler, a load of memory that does not change
+//    during the kernel, so it may be scheduled above the wait and read the
+//    buffer before the predecessor has written it.  These loads are volatile
+//    asm statements, which the compiler keeps in program order with the wait;
+//  * must not use the non-coherent path (ld.global.nc), whose contract is
+//    that the data does not change while the kernel runs.
+// The pointers they take are never declared __restrict__.
+__device__ __forceinline__ uint32_t ld_dep_u32(const void* p) {  // through L2
+  uint32_t v;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int32_t ld_dep_i32(const int32_t* p) { return static_cast<int32_t>(ld_dep_u32(p)); }
+__device__ __forceinline__ float ld_dep_f32(const float* p) { return __uint_as_float(ld_dep_u32(p)); }
+// 16 bytes, coherent and cacheable in L1 (re-read data such as the decode
+// GEMV's token codes); no memory clobber, so the compiler may still schedule
+// it freely among ordinary loads after the wait.
+__device__ __forceinline__ uint4 ld_dep_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+// 2 bytes through L2 without a memory clobber.
+__device__ __forceinline__ uint16_t ld_dep_u16_hot(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.cg.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+// 4 bytes through L2 without a memory clobber (hot loops).
+__device__ __forceinline__ uint32_t ld_dep_u32_hot(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+// 4 bytes, weak and cacheable in L1: for a few words that every warp of the
+// grid reads (the outlier mask), which through L2 alone would concentrate the
+// whole grid's requests on a handful of L2 lines.  Coherent: after the wait
+// the predecessor's writes are visible to weak loads, and none of these
+// addresses is read before it.
+__device__ __forceinline__ uint32_t ld_dep_u32_l1(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
 }
 
 // L2 prefetch of a global range (16-byte aligned address, size a multiple of 16).

@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int num_n = static_cast<int>((p.N + BN - 1) / BN);
   const int num_tiles = num_m * num_n;
   griddep_wait();  // n_out and the operands come from the preceding kernels
-  const int n_out = (p.n_out != nullptr) ? __ldcg(p.n_out) : 0;
+  int n_out = (p.n_out != nullptr) ? ld_dep_i32(p.n_out) : 0;  // clamped to [0, K] like every reader of it
+  n_out = n_out < 0 ? 0 : (n_out > p.K ? static_cast<int>(p.K) : n_out);
   const int nkb_o = (p.mode == 0) ? (n_out + 63) / 64 : 0;
   const int nkb = p.nkb_i8 + nkb_o;
   const bool has_out = nkb_o > 0;
@@ -231,11 +232,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t aph = static_cast<uint32_t>((it / nbuf) & 1);
       int m_blk, n_blk;
       tile_coords(tile, num_m, num_n, m_blk, n_blk);
-      if (!mbar_wait(&tfull_bar[buf], aph, &abort_sh, p.st, W_TFULL)) break;
-      tc_fence_after();
       const int64_t row = static_cast<int64_t>(m_blk) * BM + q * 32 + lane;
       const bool row_ok = row < p.T;
-      const float ra = (row_ok && p.mode == 0) ? __ldg(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
+      // this warp's 128 columns: lane i holds the scale and bias of column
+      // 32c + i of chunk c, loaded before the wait for the accumulators (they
+      // arrive while the MMAs run)
+      float sc4[4], bi4[4];
+      #pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int64_t col = static_cast<int64_t>(n_blk) * BN + half * 128 + c * 32 + lane;
+        const bool ok = p.mode == 0 && col < p.N;
+        sc4[c] = ok ? __ldg(&p.SCB[col]) : 0.0f;
+        bi4[c] = (ok && p.bias != nullptr) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[col]) : 0.0f;
+      }
+      const float ra = (row_ok && p.mode == 0) ? ld_dep_f32(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
+      if (!mbar_wait(&tfull_bar[buf], aph, &abort_sh, p.st, W_TFULL)) break;
+      tc_fence_after();
       #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         const int col0 = half * 128 + c * 32;
@@ -255,9 +267,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           continue;
         }
-        const int64_t my_col = gcol0 + lane;
-        const float scb_l = (my_col < p.N) ? __ldg(&p.SCB[my_col]) : 0.0f;
-        const float b_l = (p.bias != nullptr && my_col < p.N) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[my_col]) : 0.0f;
+        const float scb_l = sc4[0], b_l = bi4[0];
+        #pragma unroll
+        for (int k = 0; k < 3; ++k) {  // the next chunk's values move to slot 0
+          sc4[k] = sc4[k + 1];
+          bi4[k] = bi4[k + 1];
+        }
         uint32_t packed[16];
         #pragma unroll
         for (int i = 0; i < 32; i += 2) {

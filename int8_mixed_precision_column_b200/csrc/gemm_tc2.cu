@@ -49,7 +49,22 @@ constexpr int THREADS = 64 + NUM_EPI_WARPS * 32;
 constexpr int YST_BYTES = 32 * 32 * 2;  // one epilogue warp's 32 x 32 block of Y
 constexpr int YST_BUFS = 2;             // per warp: one filling while the other is stored
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NUM_EPI_WARPS * YST_BUFS * YST_BYTES + 1024;
-constexpr int GROUP_M = 8;  // pair tiles (256 rows) per raster group
+// Pair tiles (256 rows) per raster group: a group sweeps N with GROUP_M
+// m-blocks side by side, so each B panel is streamed once per group.
+#ifndef I8MP_PAIR_GROUP_M
+#define I8MP_PAIR_GROUP_M 8
+#endif
+constexpr int GROUP_M = I8MP_PAIR_GROUP_M;
+// L2 eviction hints: Y is written once and never read here (evict first, so
+// that it does not push the A panels a raster group re-reads out of L2);
+// optionally the A panels (X codes) are marked evict-last.
+#ifndef I8MP_Y_EVICT_FIRST
+#define I8MP_Y_EVICT_FIRST 1
+#endif
+#ifndef I8MP_A_EVICT_LAST
+#define I8MP_A_EVICT_LAST 0
+#endif
+
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_I8 = idesc_i8_s32(2 * BM, BN_MMA);
 constexpr uint16_t PAIR_MASK = 0x3;
@@ -69,8 +84,6 @@ struct Params {
   const int32_t* n_out;
   DevStatus* st;
   int mode;
-  int vec_scb;   // SCB is 16-byte aligned: a tile's 16 column scales load as 4 x float4
-  int vec_bias;  // bias is 16-byte aligned: 16 elements load as 2 x uint4
   int tma_y;     // Y leaves through shared memory by TMA stores (no extra destinations)
 };
 
@@ -145,7 +158,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   // The set-up above overlaps the tail of the row quantisation (programmatic
   // launch); n_out and every operand are read only after it has completed.
   griddep_wait();
-  const int n_out = (p.n_out != nullptr && p.mode == 0) ? __ldcg(p.n_out) : 0;
+  // n_out comes from the outlier pass (completed before the row quantisation
+  // this kernel waited for); clamped to [0, K] like every reader of it
+  int n_out = (p.n_out != nullptr && p.mode == 0) ? ld_dep_i32(p.n_out) : 0;
+  n_out = n_out < 0 ? 0 : (n_out > p.K ? static_cast<int>(p.K) : n_out);
   const int nkb_o = (n_out + 63) / 64;
   const int nkb = p.nkb_i8 + nkb_o;
   const bool has_out = nkb_o > 0;  // outlier product accumulated onto the fp32 partial outputs in TMEM
@@ -153,6 +169,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
+#if I8MP_A_EVICT_LAST
+      const uint64_t pol_a = l2_policy_evict_last();
+#endif
       int s = 0;
       uint32_t ph = 0;
       int issued[STAGES];
@@ -174,7 +193,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * STAGE_BYTES);
           const uint32_t fb = leader_smem_addr(smem_u32(&full_bar[s]));
           if (kb < p.nkb_i8) {
+#if I8MP_A_EVICT_LAST
+            tma_load_2d_pair_hint(sa, &tmA, fb, kb * BKB, row_a, pol_a);
+#else
             tma_load_2d_pair(sa, &tmA, fb, kb * BKB, row_a);
+#endif
             tma_load_2d_pair(sb, &tmB, fb, kb * BKB, row_b);
             tma_load_2d_pair(sb + BN_BOX * BKB, &tmB, fb, kb * BKB, row_b + BN_MMA);
           } else {
@@ -264,43 +287,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int half = (warp - 2) >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     int it = 0;
-    // column scales and bias of the 32 output columns from gcol0
-    auto load_scales = [&](int64_t gcol0, float (&sc)[32], float (&bi)[32]) {
-      const bool full = gcol0 + 32 <= p.N;
-      if (full && p.vec_scb) {
-        const float4* s4 = reinterpret_cast<const float4*>(p.SCB + gcol0);
-        #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 v = __ldg(s4 + q4);
-          sc[4 * q4] = v.x;
-          sc[4 * q4 + 1] = v.y;
-          sc[4 * q4 + 2] = v.z;
-          sc[4 * q4 + 3] = v.w;
-        }
-      } else {
-        #pragma unroll
-        for (int i = 0; i < 32; ++i) sc[i] = (gcol0 + i < p.N) ? __ldg(&p.SCB[gcol0 + i]) : 0.0f;
+    // Column scales and bias of this warp's 256 columns of a tile: lane i holds
+    // column 32c + i for chunk c.  They are loaded before the wait for the
+    // accumulators, so they arrive while the MMAs run; a chunk takes its 32
+    // columns' values by warp shuffles (one global round trip per tile
+    // instead of one per chunk on the epilogue's critical path).
+    float sc8[8], bi8[8];
+    auto prefetch_scales = [&](int n_blk) {
+      #pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int64_t col = static_cast<int64_t>(n_blk) * BN + half * 256 + c * 32 + lane;
+        const bool ok = col < p.N;
+        sc8[c] = ok ? __ldg(&p.SCB[col]) : 0.0f;
+        bi8[c] = (ok && p.bias != nullptr) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[col]) : 0.0f;
       }
-      if (p.bias == nullptr) {
-        #pragma unroll
-        for (int i = 0; i < 32; ++i) bi[i] = 0.0f;
-      } else if (full && p.vec_bias) {
-        const uint4* b8 = reinterpret_cast<const uint4*>(static_cast<const TE*>(p.bias) + gcol0);
-        #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          const uint4 v = __ldg(b8 + q8);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = Elem<TE>::to_float2(w[e]);
-            bi[8 * q8 + 2 * e] = f.x;
-            bi[8 * q8 + 2 * e + 1] = f.y;
-          }
-        }
-      } else {
-        #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          bi[i] = (gcol0 + i < p.N) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[gcol0 + i]) : 0.0f;
+    };
+    // the next chunk's values move to slot 0 (static register indices)
+    auto next_chunk = [&]() {
+      #pragma unroll
+      for (int c = 0; c < 7; ++c) {
+        sc8[c] = sc8[c + 1];
+        bi8[c] = bi8[c + 1];
       }
     };
     // 32 outputs of this warp's 32 rows from gcol0 (one row per lane) to Y.
@@ -308,6 +315,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // rows and columns outside Y are clipped by the store.  Otherwise direct
     // stores, to Y and its extra destinations.
     uint8_t* const ystage = smem + STAGES * STAGE_BYTES + (warp - 2) * YST_BUFS * YST_BYTES;
+#if I8MP_Y_EVICT_FIRST
+    const uint64_t pol_y = l2_policy_evict_first();
+#endif
     int ybuf = 0;
     int ystores = 0;
     auto store_y = [&](int64_t row, bool row_ok, int64_t row0, int64_t gcol0, const uint32_t (&packed)[16]) {
@@ -324,7 +334,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
+#if I8MP_Y_EVICT_FIRST
+          tma_store_2d_hint(&tmY, buf, static_cast<int32_t>(gcol0), static_cast<int32_t>(row0), pol_y);
+#else
           tma_store_2d(&tmY, buf, static_cast<int32_t>(gcol0), static_cast<int32_t>(row0));
+#endif
           bulk_commit();
         }
         ybuf ^= 1;
@@ -348,25 +362,27 @@ __global__ void __launch_bounds__(THREADS, 1)
       tile_coords(tile, num_m, num_n, m_blk, n_blk);
       const int64_t row = static_cast<int64_t>(m_blk) * 2 * BM + static_cast<int64_t>(rank) * BM + q * 32 + lane;
       const bool row_ok = row < p.T;
+      if (p.mode == 0) prefetch_scales(n_blk);
+      const float ra = (row_ok && p.mode == 0) ? ld_dep_f32(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
       if (!mbar_wait_cluster(&tfull_bar, aph, &abort_sh, p.st, W_TFULL)) break;
       tc_fence_after();
-      const float ra = (row_ok && p.mode == 0) ? __ldg(&p.sA[row]) * (1.0f / 16129.0f) : 0.0f;
       const uint32_t t_row = tmem_base + lane_base;
       if (has_out) {
         // pass 1: acc * sA * SCB / 127^2 + bias as fp32, written back in place
         #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           const int col0 = half * 256 + c * 32;
-          const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
           uint32_t acc[32];
           tmem_ld_32x32b_x32(t_row + col0, acc);
-          float sc[32], bi[32];
-          load_scales(gcol0, sc, bi);
           tmem_ld_wait();
           #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            acc[i] = __float_as_uint(fmaf(static_cast<float>(static_cast<int32_t>(acc[i])), ra * sc[i], bi[i]));
+          for (int i = 0; i < 32; ++i) {
+            const float sc = __shfl_sync(0xffffffffu, sc8[0], i);
+            const float bi = __shfl_sync(0xffffffffu, bi8[0], i);
+            acc[i] = __float_as_uint(fmaf(static_cast<float>(static_cast<int32_t>(acc[i])), ra * sc, bi));
+          }
           tmem_st_32x32b_x32(t_row + col0, acc);
+          next_chunk();
         }
         tmem_st_wait();
         tc_fence_before();
@@ -407,15 +423,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             continue;
           }
-          float sc[32], bi[32];
-          load_scales(gcol0, sc, bi);
           uint32_t packed[16];
           #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float y0 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i])), ra * sc[i], bi[i]);
-            const float y1 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i + 1])), ra * sc[i + 1], bi[i + 1]);
+            const float s0 = __shfl_sync(0xffffffffu, sc8[0], i), s1 = __shfl_sync(0xffffffffu, sc8[0], i + 1);
+            const float b0 = __shfl_sync(0xffffffffu, bi8[0], i), b1 = __shfl_sync(0xffffffffu, bi8[0], i + 1);
+            const float y0 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i])), ra * s0, b0);
+            const float y1 = fmaf(static_cast<float>(static_cast<int32_t>(acc[i + 1])), ra * s1, b1);
             packed[i >> 1] = Elem<TE>::pack2(y0, y1);
           }
+          next_chunk();
           store_y(row, row_ok, row - lane, gcol0, packed);
         }
       }
@@ -542,8 +559,6 @@ cudaError_t launch_gemm_tc2(const GemmArgs& a, cudaStream_t s) {
   p.n_out = outl ? a.n_out : nullptr;
   p.st = a.st;
   p.mode = a.mode;
-  p.vec_scb = (reinterpret_cast<uintptr_t>(a.SCB) % 16 == 0) ? 1 : 0;
-  p.vec_bias = (a.bias != nullptr && reinterpret_cast<uintptr_t>(a.bias) % 16 == 0) ? 1 : 0;
   // Y by TMA stores when it has no extra destinations and its rows are
   // 16-byte multiples (the tensor map's stride rule)
   CUtensorMap tmY = tmA;

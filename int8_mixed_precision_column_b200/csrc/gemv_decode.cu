@@ -36,6 +36,7 @@ constexpr int DV_U = 4;    // K-steps (64 B each) loaded before computing
 constexpr int DV_OB = 64;  // outlier columns staged per block
 constexpr int kPrefetchRows = 16;  // weight rows per CTA pulled into L2 before the wait
 
+
 struct DvParams {
   const int8_t* Xq;
   const float* sA;
@@ -98,7 +99,10 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
   if (threadIdx.x < kPrefetchRows && g_begin * 8 + threadIdx.x < g_end * 8)
     prefetch_l2(p.CB + (g_begin * 8 + threadIdx.x) * p.K, static_cast<uint32_t>(p.K));
   griddep_wait();
-  const int n_out = (p.mode == 0) ? __ldcg(p.n_out) : 0;
+  // Xq, sA, Xo, idx and n_out come from the prep kernel: read with the ld_dep_*
+  // loads (kept behind the wait, coherent); n_out clamped to [0, K]
+  int n_out = (p.mode == 0) ? ld_dep_i32(p.n_out) : 0;
+  n_out = n_out < 0 ? 0 : (n_out > p.K ? static_cast<int>(p.K) : n_out);
   const bool row_a = g < p.T;
   const bool row_b = g + 8 < p.T;
   const int8_t* xa_base = p.Xq + static_cast<int64_t>(g) * p.K + t4 * 16;
@@ -131,8 +135,8 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
       for (int u = 0; u < DV_U; ++u) {
         const int64_t k = (st + u) * 64;
         const bool kok = (st + u) < s_end && k + t4 * 16 < p.K;
-        xa[u] = (row_a && kok) ? __ldg(reinterpret_cast<const uint4*>(xa_base + k)) : zero4;
-        xb[u] = (row_b && kok) ? __ldg(reinterpret_cast<const uint4*>(xb_base + k)) : zero4;
+        xa[u] = (row_a && kok) ? ld_dep_v4(xa_base + k) : zero4;
+        xb[u] = (row_b && kok) ? ld_dep_v4(xb_base + k) : zero4;
       }
       #pragma unroll
       for (int u = 0; u < DV_U; ++u) {
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
         const int64_t j = g0 * 8 + r;
         float wv = 0.0f;
         if (j < g_end * 8) {
-          const int64_t col = __ldcg(&p.idx[ob + o]);
+          const int64_t col = static_cast<int32_t>(ld_dep_u32_l1(&p.idx[ob + o]));
           if (p.Wf != nullptr) {
             wv = E::to_float(static_cast<const TE*>(p.Wf)[j * p.K + col]);
           } else {
@@ -191,7 +195,8 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
       for (int e = threadIdx.x; e < kDecodeMaxT * nb; e += DV_THREADS) {
         const int t = e / nb;
         const int o = e - t * nb;
-        xo_s[t][o] = (t < p.T) ? E::to_float(static_cast<const TE*>(p.Xo)[t * p.ldo + ob + o]) : 0.0f;
+        xo_s[t][o] = (t < p.T) ? E::to_float(E::from_bits(ld_dep_u16_hot(static_cast<const TE*>(p.Xo) + t * p.ldo + ob + o)))
+                               : 0.0f;
       }
       __syncthreads();
       #pragma unroll
@@ -211,7 +216,7 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
         continue;
       }
       const float scb = __ldg(&p.SCB[j]);
-      float y = static_cast<float>(acc[h]) * (__ldg(&p.sA[tok[h]]) * (1.0f / 16129.0f) * scb) + yo[h];
+      float y = static_cast<float>(acc[h]) * (ld_dep_f32(&p.sA[tok[h]]) * (1.0f / 16129.0f) * scb) + yo[h];
       if (p.bias != nullptr) y += E::to_float(static_cast<const TE*>(p.bias)[j]);
       const int64_t off = tok[h] * p.yd.ld + j;
       const TE v = E::from_float(y);
@@ -246,6 +251,11 @@ void prefer_l1(int dev) {
 }
 
 }  // namespace
+
+void prepare_gemv_decode() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) prefer_l1(dev);
+}
 
 cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s) {
   if (a.T == 0 || a.N == 0) return cudaSuccess;

@@ -119,6 +119,18 @@ cudaError_t launch_gemv_decode(const GemmArgs& a, int num_sms, cudaStream_t s);
 
 constexpr int kDecodeMaxT = 16;
 
+// The per-device, per-process set-up the decode kernels otherwise do at their
+// first launch with a given T: whether the prep kernel's T-CTA cluster can be
+// scheduled (T = 2..kDecodeMaxT, element type `dtype`) and the GEMV's
+// shared-memory carveout hint.  Afterwards their launchers make no CUDA call
+// besides cudaGetDevice and the launch itself.
+cudaError_t prepare_prep_small(int dtype);
+void prepare_gemv_decode();
+
+// Remembers a failed CUDA result for int8_last_cuda_error() (this host
+// thread) and returns it unchanged.
+cudaError_t note_cuda_error(cudaError_t e);
+
 // Product-kernel choice (the `path` argument of the C ABI).
 enum Path : int { kPathAuto = 0, kPathTensorCore = 1, kPathDecode = 2, kPathTensorCoreSingleSM = 3 };
 

@@ -51,19 +51,25 @@ StaticLayout static_layout(int64_t T, int64_t K) {
 
 // Device address of g_scratch on the current device, resolved once per device
 // with that device current.  Host code must not use `g_scratch` itself: on the
-// host it names a stand-in object, not device memory.
+// host it names a stand-in object, not device memory.  The same first call
+// also does the decode kernels' own once-per-device set-up for every T in
+// 1..16, so that no later call makes a CUDA call other than the launches.
 i8_status scratch_for_current_device(void** addr, int* num_sms) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return I8_ERR_CUDA;
+  if (note_cuda_error(cudaGetDevice(&dev)) != cudaSuccess) return I8_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return I8_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   if (g_scratch_addr[dev] == nullptr) {
     int major = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return I8_ERR_CUDA;
+    if (note_cuda_error(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return I8_ERR_CUDA;
     if (major != 10) return I8_ERR_UNSUPPORTED;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return I8_ERR_CUDA;
+    if (note_cuda_error(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return I8_ERR_CUDA;
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return I8_ERR_CUDA;
+    if (note_cuda_error(cudaGetSymbolAddress(&p, g_scratch)) != cudaSuccess || p == nullptr) return I8_ERR_CUDA;
+    if (note_cuda_error(prepare_prep_small(kF16)) != cudaSuccess) return I8_ERR_CUDA;
+    prepare_gemv_decode();
     g_num_sms[dev] = sms;
     g_scratch_addr[dev] = p;
   }
@@ -107,7 +113,7 @@ extern "C" i8_status int8_linear_forward_decode_static(const void* X, int64_t T,
   const uint32_t hb = int8_outlier_threshold_bits(threshold);
   const cudaError_t e = launch_prep_small(X, kF16, T, K, hb, mask, mask + (K + 31) / 32, idx, n_out, Xq, sA, Xo,
                                           L.ldo, dst, stream);
-  if (e != cudaSuccess) return I8_ERR_CUDA;
+  if (note_cuda_error(e) != cudaSuccess) return I8_ERR_CUDA;
 
   GemmArgs a;
   a.Xq = Xq;
@@ -128,5 +134,5 @@ extern "C" i8_status int8_linear_forward_decode_static(const void* X, int64_t T,
   a.K = K;
   a.mode = 0;
   a.pdl = true;  // follows the prep kernel
-  return launch_gemv_decode(a, num_sms, stream) == cudaSuccess ? I8_OK : I8_ERR_CUDA;
+  return note_cuda_error(launch_gemv_decode(a, num_sms, stream)) == cudaSuccess ? I8_OK : I8_ERR_CUDA;
 }

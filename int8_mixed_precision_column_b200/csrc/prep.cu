@@ -144,7 +144,7 @@ __device__ __forceinline__ uint32_t flag_bits8(const uint4& v, uint32_t h2) {
 template <typename TE>
 __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const TE* __restrict__ X, int64_t T, int64_t K,
                                                                     uint32_t hbits, int wc, int64_t rows_per_cta,
-                                                                    uint32_t* __restrict__ mask,
+                                                                    uint32_t* mask,
                                                                     uint32_t* __restrict__ prefix, int32_t* __restrict__ idx,
                                                                     int32_t* __restrict__ n_out, DevStatus* st) {
   __shared__ int s_last;
@@ -198,11 +198,11 @@ __global__ void __launch_bounds__(kMaskThreads) outlier_mask_kernel(const TE* __
   const int64_t w0 = threadIdx.x * per;
   const int64_t w1 = min(nwords, w0 + per);
   int cnt = 0;
-  for (int64_t w = w0; w < w1; ++w) cnt += __popc(__ldcg(&mask[w]));
+  for (int64_t w = w0; w < w1; ++w) cnt += __popc(ld_dep_u32(&mask[w]));
   int total = 0;
   int pos = block_exclusive_scan<kMaskThreads>(cnt, s_scan, &total);
   for (int64_t w = w0; w < w1; ++w) {
-    uint32_t m = __ldcg(&mask[w]);
+    uint32_t m = ld_dep_u32(&mask[w]);
     prefix[w] = static_cast<uint32_t>(pos);
     while (m) {
       const int b = __ffs(m) - 1;
@@ -264,10 +264,18 @@ constexpr int kRowWarps = kRowThreads / 32;
 constexpr int kRowUnroll = 8;
 
 // The outlier pass's outputs (mask, prefix, idx, n_out) decide addresses in the
-// kernels that follow it under programmatic launch: those kernels read them
-// through L2 (ld.global.cg), never through the non-coherent read-only path.
+// kernels that follow it under programmatic launch.  Those kernels read them
+// with the ld_dep_* loads (kept behind the programmatic wait, through L2) and
+// take them through pointers without __restrict__; n_out is also clamped to
+// [0, K], so that no value it could hold turns into an address outside the
+// workspace.
 __device__ __forceinline__ uint32_t mask_byte(const uint32_t* mask, int64_t chunk) {
-  return (__ldcg(&mask[chunk >> 2]) >> ((chunk & 3) * 8)) & 0xffu;
+  return (ld_dep_u32_l1(&mask[chunk >> 2]) >> ((chunk & 3) * 8)) & 0xffu;
+}
+
+__device__ __forceinline__ int load_n_out(const int32_t* n_out_p, int64_t K) {
+  const int32_t n = ld_dep_i32(n_out_p);
+  return static_cast<int>(n < 0 ? 0 : (n > K ? K : n));
 }
 
 // Largest magnitude pattern among the non-outlier elements of a chunk.
@@ -330,8 +338,8 @@ template <typename TE, bool kShared = false>
 __device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, int64_t chunk, const uint32_t* mask,
                                                  const uint32_t* prefix, TE* xo_row) {
   const TE* h = reinterpret_cast<const TE*>(&v);
-  const uint32_t mw = kShared ? mask[chunk >> 2] : __ldcg(&mask[chunk >> 2]);
-  const uint32_t base = kShared ? prefix[chunk >> 2] : __ldcg(&prefix[chunk >> 2]);
+  const uint32_t mw = kShared ? mask[chunk >> 2] : ld_dep_u32_l1(&mask[chunk >> 2]);
+  const uint32_t base = kShared ? prefix[chunk >> 2] : ld_dep_u32_l1(&prefix[chunk >> 2]);
   const int sh = static_cast<int>(chunk & 3) * 8;
   const uint32_t first = base + __popc(mw & ((1u << sh) - 1u));
   if (mb == 0xffu && (first & 7u) == 0) {
@@ -350,13 +358,22 @@ __device__ __forceinline__ void scatter_outliers(const uint4& v, uint32_t mb, in
 // groups of L = min(32, npad/8 rounded up to a power of two) lanes per row,
 // each lane builds 8 consecutive outputs and writes them with one 16-byte
 // store (npad is a multiple of 64, ldo of 64: rows stay 16-byte aligned).
+// idx entries a Wo-gather CTA keeps in shared memory: every warp of the
+// gather reads the same few idx words, which through L2 alone would put all
+// of the grid's requests on one or two L2 lines.
+constexpr int kWoIdx = 2048;
+
 template <typename TE, int NT>
 __device__ __forceinline__ void wo_gather(int64_t wblk, int64_t wo_blocks, int n_out, int64_t npad,
-                                          const int32_t* __restrict__ idx, const int8_t* __restrict__ CB,
+                                          const int32_t* idx, const int8_t* __restrict__ CB,
                                           const float* __restrict__ SCB, int64_t N, int64_t K, TE* __restrict__ Wo,
                                           int64_t ldo, const TE* __restrict__ Wf) {
   using E = Elem<TE>;
-  if (n_out == 0) return;
+  __shared__ int32_t s_idx[kWoIdx];
+  if (n_out == 0) return;  // n_out is the same for every thread of the grid
+  const int n_staged = n_out < kWoIdx ? n_out : kWoIdx;
+  for (int o = threadIdx.x; o < n_staged; o += NT) s_idx[o] = ld_dep_i32(&idx[o]);
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int chunks = static_cast<int>(npad / 8);
   int lpr_log = 0;  // log2 of lanes per row
@@ -383,7 +400,7 @@ __device__ __forceinline__ void wo_gather(int64_t wblk, int64_t wo_blocks, int n
           const int o = o0 + i + h;
           f[h] = 0.0f;
           if (o < n_out) {
-            const int col = __ldcg(&idx[o]);
+            const int col = o < kWoIdx ? s_idx[o] : static_cast<int>(ld_dep_u32_l1(&idx[o]));
             f[h] = wfrow != nullptr ? E::to_float(wfrow[col])
                                     : __fdiv_rn(__fmul_rn(static_cast<float>(__ldg(&cbrow[col])), scb), 127.0f);
           }
@@ -397,8 +414,8 @@ __device__ __forceinline__ void wo_gather(int64_t wblk, int64_t wo_blocks, int n
 
 template <typename TE>
 __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
-    const TE* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
-    const uint32_t* __restrict__ prefix, const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p,
+    const TE* __restrict__ X, int64_t T, int64_t K, const uint32_t* mask, const uint32_t* prefix,
+    const int32_t* idx, const int32_t* n_out_p,
     int8_t* __restrict__ Xq, float* __restrict__ sA, TE* __restrict__ Xo, int64_t ldo,
     const int8_t* __restrict__ CB, const float* __restrict__ SCB, int64_t N, TE* __restrict__ Wo,
     const TE* __restrict__ Wf, int64_t row_blocks, int64_t wo_blocks) {
@@ -406,7 +423,7 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(
   const int lane = threadIdx.x & 31;
   griddep_launch_dependents();
   griddep_wait();  // mask, prefix, idx, n_out come from the outlier pass
-  const int n_out = __ldcg(n_out_p);
+  const int n_out = load_n_out(n_out_p, K);
   const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
 
   if (static_cast<int64_t>(blockIdx.x) >= row_blocks) {
@@ -476,8 +493,8 @@ constexpr int64_t kResidentMaxK = static_cast<int64_t>(kRowCtaThreads) * kRowCta
 // flight (R > 1 only when the row fits the S threads x 8 chunks).
 template <typename TE, bool kResident>
 __global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
-    const TE* __restrict__ X, int64_t T, int64_t K, const uint32_t* __restrict__ mask,
-    const uint32_t* __restrict__ prefix, const int32_t* __restrict__ idx, const int32_t* __restrict__ n_out_p,
+    const TE* __restrict__ X, int64_t T, int64_t K, const uint32_t* mask, const uint32_t* prefix,
+    const int32_t* idx, const int32_t* n_out_p,
     int8_t* __restrict__ Xq, float* __restrict__ sA, TE* __restrict__ Xo, int64_t ldo,
     const int8_t* __restrict__ CB, const float* __restrict__ SCB, int64_t N, TE* __restrict__ Wo,
     const TE* __restrict__ Wf, int64_t row_blocks, int64_t wo_blocks, int rpc_log) {
@@ -485,7 +502,7 @@ __global__ void __launch_bounds__(kRowCtaThreads) rowquant_cta_kernel(
   __shared__ uint32_t s_max[kRowCtaThreads / 32];
   griddep_launch_dependents();
   griddep_wait();  // mask, prefix, idx, n_out come from the outlier pass
-  const int n_out = __ldcg(n_out_p);
+  const int n_out = load_n_out(n_out_p, K);
   const int64_t npad = ((static_cast<int64_t>(n_out) + 63) / 64) * 64;
   if (static_cast<int64_t>(blockIdx.x) >= row_blocks) {
     wo_gather<TE, kRowCtaThreads>(static_cast<int64_t>(blockIdx.x) - row_blocks, wo_blocks, n_out, npad, idx, CB,
@@ -787,6 +804,19 @@ bool cluster_form_ok(int64_t T, int et) {
   if (!ok) (void)cudaGetLastError();  // a refused opt-in or query only means: no cluster form
   c = ok ? 1 : -1;
   return ok;
+}
+
+cudaError_t prepare_prep_small(int dtype) {
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  for (int64_t T = 2; T <= kDecodeMaxT; ++T) {
+    if (dtype == kBF16)
+      (void)cluster_form_ok<__nv_bfloat16>(T, 1);
+    else
+      (void)cluster_form_ok<__half>(T, 0);
+  }
+  return cudaSuccess;
 }
 
 template <typename TE>

@@ -30,8 +30,8 @@ extern "C" i8_status int8_selftest_wait_timeout(void* workspace, size_t workspac
       workspace_bytes < sizeof(DevStatus))
     return I8_ERR_WORKSPACE;
   if (limit_us == 0 || limit_us > 2000000) return I8_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(workspace, 0, sizeof(DevStatus), stream) != cudaSuccess) return I8_ERR_CUDA;
+  if (note_cuda_error(cudaMemsetAsync(workspace, 0, sizeof(DevStatus), stream)) != cudaSuccess) return I8_ERR_CUDA;
   wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(static_cast<DevStatus*>(workspace),
                                                   static_cast<uint64_t>(limit_us) * 1000ull);
-  return cudaGetLastError() == cudaSuccess ? I8_OK : I8_ERR_CUDA;
+  return note_cuda_error(cudaGetLastError()) == cudaSuccess ? I8_OK : I8_ERR_CUDA;
 }
