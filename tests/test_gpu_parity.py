@@ -344,9 +344,25 @@ def test_bloom_ffn_up_decode(T):
 
 
 def test_bloom_ffn_up_prefill_sampled():
+    """The headline config at full size (T=8192, K=14336, N=57344): every stage
+    on sampled rows and columns that touch every output tile; then the int32
+    accumulators of the pair kernel over the whole [8192, 57344] output (the
+    same 256 x 512 tiles, persistent grid and raster as the forward, int32
+    epilogue), bit for bit against the oracle's exact int8 product on 2 rows of
+    every 128-row block and all 57344 columns, and CB bit for bit on every
+    row of W."""
     p = workloads.bloom_ffn_up_prefill(8192, seed=0, device="cuda")
     g = gpu_forward(p, "auto")
-    check_forward(p, g, rows=tile_rows(p.T, per_tile=2), cols=tile_cols(p.N, per_tile=8))
+    rows = tile_rows(p.T, per_tile=2)
+    r = check_forward(p, g, rows=rows, cols=tile_cols(p.N, per_tile=8))
+    acc = native.int8_gemm_i32(g["Xq"], g["CB"], path=PATHS["tc"])
+    acc_rows = to_np(acc[torch.as_tensor(rows, device="cuda")])
+    del acc
+    chunk = 4096
+    for j0 in range(0, p.N, chunk):
+        CBo, _ = O.quantize_weight(p.W[j0: j0 + chunk].cpu().numpy())
+        assert np.array_equal(to_np(g["CB"][j0: j0 + chunk]), CBo), j0
+        assert np.array_equal(acc_rows[:, j0: j0 + chunk], O.int8_matmul(r["Xq"], CBo)), j0
 
 
 def test_host_buffer_forward_matches_device_forward():

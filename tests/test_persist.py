@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import llm_int8 as O
 from int8_mixed_precision_column_b200 import build, native, workloads
 
 
@@ -75,14 +76,30 @@ def test_malformed_images_are_rejected():
 
 
 @pytest.mark.gpu
-def test_loaded_layer_gives_the_same_forward(tmp_path):
+@pytest.mark.parametrize("path", [native.PATH_AUTO, native.PATH_DECODE])
+def test_loaded_layer_matches_the_oracle(tmp_path, path):
+    """A layer saved and loaded back: its CB/SCB equal the oracle's quantisation
+    of the fp16 weight bit for bit, and its forward matches the oracle's Y at
+    the fp16 tolerance (and the forward of the layer before saving bit for bit)."""
     assert torch.cuda.is_available()
-    p = workloads.make_problem("persist", 64, 1024, 512, n_planted=5, bias_std=0.01, seed=3)
+    T = 64 if path == native.PATH_AUTO else 16
+    p = workloads.make_problem("persist", T, 1024, 512, n_planted=5, bias_std=0.01, seed=3)
     CB, SCB = native.int8_quantize_weight(p.W.cuda())
     bias = p.bias.cuda()
-    path = tmp_path / "layer.i8mp"
-    native.save_quantized(str(path), CB, SCB, bias)
-    CB2, SCB2, b2 = native.load_quantized(str(path), device="cuda")
-    Y1, idx1, n1, _ = native.int8_linear_forward(p.X.cuda(), CB, SCB, bias, 6.0)
-    Y2, idx2, n2, _ = native.int8_linear_forward(p.X.cuda(), CB2, SCB2, b2, 6.0)
-    assert torch.equal(Y1, Y2) and int(n1) == int(n2)
+    f = tmp_path / "layer.i8mp"
+    native.save_quantized(str(f), CB, SCB, bias)
+    del CB, SCB
+    CB2, SCB2, b2 = native.load_quantized(str(f), device="cuda")
+    CBo, SCBo = O.quantize_weight(p.W.numpy())
+    assert np.array_equal(CB2.cpu().numpy(), CBo) and np.array_equal(SCB2.cpu().numpy(), SCBo)
+    assert torch.equal(b2.cpu(), p.bias)
+    Y2, idx2, n2, ws = native.int8_linear_forward(p.X.cuda(), CB2, SCB2, b2, 6.0, path=path)
+    assert native.int8_check_status(ws)[0] == 0
+    r = O.linear_forward(p.X.numpy(), CBo, SCBo, p.bias.numpy(), 6.0)
+    n = int(n2.item())
+    assert n == r["n_out"] and np.array_equal(idx2[:n].cpu().numpy(), r["idx"])
+    err = np.abs(Y2.cpu().numpy().astype(np.float64) - r["Y"]).max()
+    assert err <= O.y_tolerance(r["Y"]), err
+    Y1, _, _, _ = native.int8_linear_forward(p.X.cuda(), torch.from_numpy(CBo).cuda(), torch.from_numpy(SCBo).cuda(),
+                                             bias, 6.0, path=path)
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
