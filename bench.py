@@ -12,8 +12,8 @@ Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
 Under torchrun (N > 1) every rank runs an independent problem of the same
 shape (weak scaling; no data-path collective); the reported time is the max
 over ranks and the value is the work of all ranks divided by it.
-``--impl reference`` times the CPU oracle (a deliberately plain numpy
-restatement of the method) on a bounded sample of the same workload.
+``--impl reference`` times the CPU oracle (the plain C++ restatement of the
+method, one thread per core) on a bounded sample of the same workload.
 """
 
 from __future__ import annotations
@@ -372,6 +372,87 @@ def run_e2e(args, X, CB, SCB, bias, threshold, T, K, N, world, dev) -> dict:
                          "api": "int8_linear_forward_host (one step at a time)"}}
 
 
+DECODE_TOKENS = (1, 4, 16)
+
+
+def run_decode_lines(args, rank, world, dev) -> dict:
+    """The HBM-bound half of the metric: BLOOM-176B FFN-up decode forwards
+    (X [T, 14336] with 8 outlier dims, W [57344, 14336] as int8 CB/SCB) for
+    T in 1, 4, 16, each timed like the headline workload: CB (822 MB) is
+    larger than L2, so steps run back to back without a flush (a flush by
+    writing a scratch buffer would leave L2 full of dirty lines that the next
+    step has to write back), timed by CUDA events around all steps, max over
+    ranks."""
+    from int8_mixed_precision_column_b200 import native
+
+    peaks, peak_src = load_peaks()
+    lines = {}
+    sampler = ClockSampler(pci_bus_id(dev))
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.5)
+    sampler.mark_begin()
+    for T in DECODE_TOKENS:
+        p = workloads.bloom_ffn_up_decode(T, seed=rank_seed(rank), device="cuda")
+        K, N = p.K, p.N
+        CB, SCB = native.int8_quantize_weight(p.W)
+        del p.W
+        X, bias = p.X, p.bias
+        Y = torch.empty((T, N), dtype=torch.float16, device=dev)
+        idx = torch.empty((K,), dtype=torch.int32, device=dev)
+        n_out = torch.empty((1,), dtype=torch.int32, device=dev)
+        ws = native.new_workspace(T, K, N, dev)
+        for _ in range(args.warmup):
+            native.int8_linear_forward(X, CB, SCB, bias, p.threshold, Y=Y, idx=idx, n_out=n_out, workspace=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record()
+        for i in range(args.steps):
+            native.int8_linear_forward(X, CB, SCB, bias, p.threshold, Y=Y, idx=idx, n_out=n_out, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        st, where = native.int8_check_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status {native.int8_status_string(st)} at {where:#x}")
+        ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
+        nstage = max(3, min(args.steps, 20))
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nstage)]
+        for row in ev:
+            for e in row:
+                e.record()
+        for i in range(nstage):
+            native.int8_linear_forward_timed(X, CB, SCB, bias, p.threshold, Y, idx, n_out, ws, ev[i])
+        torch.cuda.synchronize()
+        prep_ms = reduce_max(statistics.mean(e[0].elapsed_time(e[2]) for e in ev), world, dev)
+        prod_ms = reduce_max(statistics.mean(e[2].elapsed_time(e[3]) for e in ev), world, dev)
+        n_o = int(n_out.item())
+        work = algorithmic_work(T, K, N, n_o)
+        step_gbs = work["product_bytes"] / (ms * 1e-3) / 1e9
+        prod_gbs = work["product_bytes"] / (prod_ms * 1e-3) / 1e9
+        lines[f"T{T}"] = {
+            "workload": f"bloom176b_ffn_up_decode_T{T}", "T": T, "K": K, "N": N, "n_out": n_o,
+            "ms_per_step": ms, "tokens_per_s": T * world / (ms * 1e-3),
+            "TOPS": work["int8_ops"] * world / (ms * 1e-3) / 1e12,
+            "algorithmic_bytes_per_step": work["product_bytes"],
+            "GBps": step_gbs, "frac_of_hbm": step_gbs / peaks["hbm_gbs"],
+            "stage_ms": {"prep": prep_ms, "product": prod_ms},
+            "product_kernel": {"kernel": "gemv_i8_decode_kernel", "GBps": prod_gbs,
+                               "frac_of_hbm": prod_gbs / peaks["hbm_gbs"]},
+        }
+        del CB, SCB, X, Y, ws, p
+        torch.cuda.empty_cache()
+    sampler.mark_end()
+    clocks = sampler.stop() if rank == 0 else None
+    return {"note": "BLOOM-176B FFN-up decode, whole forward (one-kernel prep + weight-streaming GEMV) per step; "
+                    "bytes = CB + SCB + bias + X codes + Y (the algorithmic HBM traffic); inputs larger than L2 "
+                    "(no flush); stage_ms from a separate pass with events between the kernels",
+            "peak": peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs (copy)", "lines": lines,
+            "clocks": clocks}
+
+
 def run_ours(args, rank, world, local_rank) -> dict | None:
     from int8_mixed_precision_column_b200 import build, native
 
@@ -401,7 +482,15 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     ws = native.new_workspace(T, K, N, dev)
     working_set = T * K * 3 + N * K + T * N * 2
     flush = working_set < 2 * L2_BYTES
+    # L2 flush between steps: write a buffer twice the size of L2, then read
+    # another one, so that L2 holds clean lines of neither the workload nor
+    # the flush (dirty flush lines would be written back during the timed step)
     scrub = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
+    scrub_ro = torch.ones(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
+
+    def flush_l2():
+        scrub.add_(1)
+        scrub_ro.sum()
 
     nsteps = args.steps
     # Steps are timed as plain forwards (the kernels chain by programmatic
@@ -422,7 +511,7 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
 
     for i in range(args.warmup):
         if flush:
-            scrub.add_(1)
+            flush_l2()
         step()
     torch.cuda.synchronize()
     st, where = native.int8_check_status(ws)
@@ -440,7 +529,7 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     outer[0].record()
     for i in range(nsteps):
         if flush:
-            scrub.add_(1)
+            flush_l2()
         bounds[i][0].record()
         step()
         bounds[i][1].record()
@@ -458,7 +547,7 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
 
     for i in range(nstage):
         if flush:
-            scrub.add_(1)
+            flush_l2()
         native.int8_linear_forward_timed(X, CB, SCB, bias, p.threshold, Y, idx, n_out, ws, ev[i], path=args.path)
     torch.cuda.synchronize()
     st, where = native.int8_check_status(ws)
@@ -471,9 +560,17 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     # end to end through the host-buffer entry points: pinned X in, Y/idx/n_out out, every step
     e2e = None
     if not args.no_e2e and elem == torch.float16:  # the blocking host entry point takes fp16
-        del ws
+        ws = None
         torch.cuda.empty_cache()
         e2e = run_e2e(args, X, CB, SCB, bias, p.threshold, T, K, N, world, dev)
+
+    decode_lines = None
+    if args.workload == DEFAULT_WORKLOAD and not args.no_decode and elem == torch.float16:
+        # the headline workload's buffers are released before the decode layers are built
+        X = Y = idx = n_out = CB = SCB = scrub = scrub_ro = ws = bias = None
+        p.X = p.bias = None
+        torch.cuda.empty_cache()
+        decode_lines = run_decode_lines(args, rank, world, dev)
 
     if rank != 0:
         return None
@@ -528,7 +625,8 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
         "config": {"workload": args.workload, "T": T, "K": K, "N": N, "threshold": p.threshold, "path": args.path,
                    "elem": args.dtype,
                    "n_out": n_outliers, "parallelism": f"independent problem per rank x{world}",
-                   "l2": "L2 flushed between steps" if flush else "inputs larger than L2 (no flush)"},
+                   "l2": ("L2 flushed between steps (write 252 MB, then read 252 MB)" if flush
+                          else "inputs larger than L2 (no flush)")},
         "stage_ms_note": "per-stage CUDA events from a separate pass with events between the kernels "
                          "(no programmatic overlap there); value and ms_per_step time plain forwards",
         "stage_ms": {"outliers": statistics.mean(outl_ms), "rowquant": statistics.mean(rowq_ms),
@@ -539,6 +637,8 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
         "e2e": e2e,
         "device": torch.cuda.get_device_name(dev),
     }
+    if decode_lines is not None:
+        out["decode"] = decode_lines
     if cpu_sample is not None:
         out["cpu_baseline"] = cpu_baseline(cpu_sample, p.threshold, seconds=args.cpu_seconds)
     return out
@@ -560,21 +660,25 @@ def sample_problem(p, rows: int, cols: int):
     return X, W, b
 
 
-def blas_threads() -> int:
+def host_threads() -> int:
+    """Cores this process may run on (the C++ oracle starts one thread per core)."""
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
-    except Exception:
-        pass
-    return os.cpu_count() or 1
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpp_oracle():
+    """The plain C++ oracle (oracle/llm_int8_ref.cpp), one thread per host core."""
+    from oracle import cpp
+
+    cpp.build()
+    return cpp.Oracle(threads=host_threads())
 
 
 def oracle_rate(X, W, b, thr, seconds: float) -> tuple[float, int, float]:
-    """Run the oracle forward on (X, W) repeatedly for ~`seconds`; returns (TOPS, reps, s/rep)."""
-    from oracle import llm_int8 as O
-
+    """Run the C++ oracle's forward on (X, W) repeatedly for ~`seconds`; returns (TOPS, reps, s/rep)."""
+    O = cpp_oracle()
     CB, SCB = O.quantize_weight(W)  # layer set-up, not part of a step
     T, K = X.shape
     N = W.shape[0]
@@ -591,9 +695,10 @@ def oracle_rate(X, W, b, thr, seconds: float) -> tuple[float, int, float]:
 def cpu_baseline(sample, threshold: float, seconds: float = 12.0) -> dict:
     X, W, b = sample
     v, reps, per = oracle_rate(X, W, b, threshold, seconds)
-    return {"value": v, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"full oracle forward on {X.shape[0]} token rows x {W.shape[0]} output features of the "
-                      f"workload (K={X.shape[1]}), repeated {reps}x ({per:.2f} s each)"}
+    return {"value": v, "unit": "TOPS", "cores": host_threads(), "kind": "oracle",
+            "sample": f"full forward of the plain C++ oracle (every stage, plain loops, one thread per core) on "
+                      f"{X.shape[0]} token rows x {W.shape[0]} output features of the workload (K={X.shape[1]}), "
+                      f"repeated {reps}x ({per:.2f} s each)"}
 
 
 def run_reference(args, rank, world, local_rank) -> dict | None:
@@ -602,8 +707,7 @@ def run_reference(args, rank, world, local_rank) -> dict | None:
     p = WORKLOADS[args.workload]("cpu", 0)
     T, K, N = p.T, p.K, p.N
     X, W, b = sample_problem(p, rows=64, cols=2048)
-    from oracle import llm_int8 as O
-
+    O = cpp_oracle()
     CB, SCB = O.quantize_weight(W)
     for _ in range(args.warmup):
         O.linear_forward(X, CB, SCB, b, p.threshold)
@@ -614,15 +718,15 @@ def run_reference(args, rank, world, local_rank) -> dict | None:
     ms = el / args.steps * 1e3
     ops = 2.0 * X.shape[0] * W.shape[0] * K
     v = ops / (ms * 1e-3) / 1e12
-    sample = (f"oracle forward on {X.shape[0]} token rows x {W.shape[0]} output features of the workload "
-              f"(T={T}, K={K}, N={N}) per step")
+    sample = (f"plain C++ oracle forward on {X.shape[0]} token rows x {W.shape[0]} output features of the "
+              f"workload (T={T}, K={K}, N={N}) per step")
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TOPS",
             "tokens_per_s": X.shape[0] / (ms * 1e-3), "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8 codes, fp64 reference arithmetic (numpy)",
+            "vs_baseline": None, "dtype": "int8 codes, int64 dot products, fp64 reference arithmetic (plain C++)",
             "data": "synthetic (seeded)",
             "config": {"workload": args.workload, "T": T, "K": K, "N": N, "threshold": p.threshold},
-            "cpu_baseline": {"value": v, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": v, "unit": "TOPS", "cores": host_threads(), "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -644,6 +748,8 @@ def main() -> None:
     ap.add_argument("--shard-n", action="store_true",
                     help="split one layer along N over the ranks (strong scaling; Y gathered by peer stores)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the BLOOM FFN-up decode lines the default workload's line carries")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
