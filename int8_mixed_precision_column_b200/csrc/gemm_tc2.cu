@@ -23,10 +23,13 @@
 // output acc * sA * SCB / 127^2 + bias (tcgen05.st), the leader then issues
 // the kind::f16 MMAs over the outlier columns accumulating onto it, and a
 // second epilogue pass converts to the 16-bit output.
-// Y leaves by TMA stores: each epilogue warp packs its 32 x 32 block into one
-// of two 2 KB shared-memory buffers and issues one tiled store (32 scattered
-// 16-byte stores per instruction before; 2 % faster).  With extra
-// destinations (the N-sharded forward) the epilogue stores directly.
+// Epilogue: 16 warps per CTA, 4 per TMEM lane quarter, each owning 32 rows
+// x 128 columns (4 chunks of 32): a warp's chunks run one after another, and
+// 16 warps measured 5 % faster than 8 at the Llama width, 1-2.5 % at the
+// BLOOM and density-sweep shapes.  Y leaves by TMA stores: each epilogue warp
+// packs its 32 x 32 block into its 2 KB shared-memory buffer and issues one
+// tiled store.  With extra destinations (the N-sharded forward) the epilogue
+// stores directly.
 // No TMA load uses cluster multicast: each CTA loads its own halves.
 #include <cuda.h>
 
@@ -44,15 +47,26 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BKB;       // 16 KB
 constexpr int B_BYTES = 2 * BN_BOX * BKB;  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_EPI_WARPS = 8;
+// Epilogue warps per CTA: 4 per TMEM lane quarter with 16 (each owning 128
+// columns, 4 chunks of 32) or 2 with 8 (256 columns, 8 chunks).  A warp's
+// chunks run one after another, so more warps shorten the epilogue.
+#ifndef I8MP_PAIR_EPI_WARPS
+#define I8MP_PAIR_EPI_WARPS 16
+#endif
+constexpr int NUM_EPI_WARPS = I8MP_PAIR_EPI_WARPS;
+static_assert(NUM_EPI_WARPS == 8 || NUM_EPI_WARPS == 16, "2 or 4 epilogue warps per TMEM lane quarter");
+constexpr int EPI_COLS = BN / (NUM_EPI_WARPS / 4);  // output columns per epilogue warp
+constexpr int EPI_CHUNKS = EPI_COLS / 32;
 constexpr int THREADS = 64 + NUM_EPI_WARPS * 32;
 constexpr int YST_BYTES = 32 * 32 * 2;  // one epilogue warp's 32 x 32 block of Y
-constexpr int YST_BUFS = 2;             // per warp: one filling while the other is stored
+// staging buffers per warp: with 8 warps one fills while the other is
+// stored; with 16, one (shared memory holds no more beside 4 stages)
+constexpr int YST_BUFS = NUM_EPI_WARPS == 8 ? 2 : 1;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NUM_EPI_WARPS * YST_BUFS * YST_BYTES + 1024;
 // Pair tiles (256 rows) per raster group: a group sweeps N with GROUP_M
 // m-blocks side by side, so each B panel is streamed once per group.
 #ifndef I8MP_PAIR_GROUP_M
-#define I8MP_PAIR_GROUP_M 8
+#define I8MP_PAIR_GROUP_M 16
 #endif
 constexpr int GROUP_M = I8MP_PAIR_GROUP_M;
 // L2 eviction hints: Y is written once and never read here (evict first, so
@@ -284,19 +298,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - 2) >> 2;  // which EPI_COLS-column group of the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     int it = 0;
-    // Column scales and bias of this warp's 256 columns of a tile: lane i holds
+    // Column scales and bias of this warp's EPI_COLS columns of a tile: lane i holds
     // column 32c + i for chunk c.  They are loaded before the wait for the
     // accumulators, so they arrive while the MMAs run; a chunk takes its 32
     // columns' values by warp shuffles (one global round trip per tile
     // instead of one per chunk on the epilogue's critical path).
-    float sc8[8], bi8[8];
+    float sc8[EPI_CHUNKS], bi8[EPI_CHUNKS];
     auto prefetch_scales = [&](int n_blk) {
       #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int64_t col = static_cast<int64_t>(n_blk) * BN + half * 256 + c * 32 + lane;
+      for (int c = 0; c < EPI_CHUNKS; ++c) {
+        const int64_t col = static_cast<int64_t>(n_blk) * BN + half * EPI_COLS + c * 32 + lane;
         const bool ok = col < p.N;
         sc8[c] = ok ? __ldg(&p.SCB[col]) : 0.0f;
         bi8[c] = (ok && p.bias != nullptr) ? Elem<TE>::to_float(static_cast<const TE*>(p.bias)[col]) : 0.0f;
@@ -305,7 +319,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // the next chunk's values move to slot 0 (static register indices)
     auto next_chunk = [&]() {
       #pragma unroll
-      for (int c = 0; c < 7; ++c) {
+      for (int c = 0; c < EPI_CHUNKS - 1; ++c) {
         sc8[c] = sc8[c + 1];
         bi8[c] = bi8[c + 1];
       }
@@ -341,7 +355,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #endif
           bulk_commit();
         }
-        ybuf ^= 1;
+        ybuf = ybuf + 1 == YST_BUFS ? 0 : ybuf + 1;  // stays within this warp's YST_BUFS buffers
         ++ystores;
         return;
       }
@@ -370,8 +384,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (has_out) {
         // pass 1: acc * sA * SCB / 127^2 + bias as fp32, written back in place
         #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          const int col0 = half * 256 + c * 32;
+        for (int c = 0; c < EPI_CHUNKS; ++c) {
+          const int col0 = half * EPI_COLS + c * 32;
           uint32_t acc[32];
           tmem_ld_32x32b_x32(t_row + col0, acc);
           tmem_ld_wait();
@@ -392,8 +406,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         // pass 2: the outlier product has been added; convert and store
         #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          const int col0 = half * 256 + c * 32;
+        for (int c = 0; c < EPI_CHUNKS; ++c) {
+          const int col0 = half * EPI_COLS + c * 32;
           const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
           uint32_t yv[32];
           tmem_ld_32x32b_x32(t_row + col0, yv);
@@ -406,8 +420,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       } else {
         #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          const int col0 = half * 256 + c * 32;
+        for (int c = 0; c < EPI_CHUNKS; ++c) {
+          const int col0 = half * EPI_COLS + c * 32;
           const int64_t gcol0 = static_cast<int64_t>(n_blk) * BN + col0;
           uint32_t acc[32];
           tmem_ld_32x32b_x32(t_row + col0, acc);
