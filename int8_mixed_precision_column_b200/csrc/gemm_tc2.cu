@@ -170,15 +170,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem_base = tmem_base_sh;
 
   // The set-up above overlaps the tail of the row quantisation (programmatic
-  // launch); n_out and every operand are read only after it has completed.
-  griddep_wait();
-  // n_out comes from the outlier pass (completed before the row quantisation
-  // this kernel waited for); clamped to [0, K] like every reader of it
-  int n_out = (p.n_out != nullptr && p.mode == 0) ? ld_dep_i32(p.n_out) : 0;
-  n_out = n_out < 0 ? 0 : (n_out > p.K ? static_cast<int>(p.K) : n_out);
-  const int nkb_o = (n_out + 63) / 64;
-  const int nkb = p.nkb_i8 + nkb_o;
-  const bool has_out = nkb_o > 0;  // outlier product accumulated onto the fp32 partial outputs in TMEM
+  // launch).  Every read of what the preceding kernels wrote (A, sA, n_out,
+  // the outlier operands) follows griddepcontrol.wait in the role that makes
+  // it; CB, SCB and bias are not written by them.
+  // Outlier K-blocks: n_out comes from the outlier pass (completed before the
+  // row quantisation this kernel waits for); clamped to [0, K] like every
+  // reader of it.
+  auto outlier_kblocks = [&]() -> int {
+    int n_out = (p.n_out != nullptr && p.mode == 0) ? ld_dep_i32(p.n_out) : 0;
+    n_out = n_out < 0 ? 0 : (n_out > p.K ? static_cast<int>(p.K) : n_out);
+    return (n_out + 63) / 64;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer (both CTAs)
@@ -191,34 +193,66 @@ __global__ void __launch_bounds__(THREADS, 1)
       int issued[STAGES];
       #pragma unroll
       for (int i = 0; i < STAGES; ++i) issued[i] = 0;
+      // The B halves (CB) of the first tile's first K-blocks go out before the
+      // wait: the stages are fresh, and CB is not an output of the preceding
+      // kernels.  Their A halves follow the wait.
+      int pre = 0;
+      if (pair < num_tiles) {
+        int m_blk, n_blk;
+        tile_coords(pair, num_m, num_n, m_blk, n_blk);
+        const int row_b = n_blk * BN + static_cast<int>(rank) * BN_BOX;
+        pre = p.nkb_i8 < STAGES ? p.nkb_i8 : STAGES;
+        for (int kb = 0; kb < pre; ++kb) {
+          uint8_t* sb = smem + kb * STAGE_BYTES + A_BYTES;
+          if (leader) mbar_arrive_expect_tx(&full_bar[kb], 2 * STAGE_BYTES);
+          const uint32_t fb = leader_smem_addr(smem_u32(&full_bar[kb]));
+          tma_load_2d_pair(sb, &tmB, fb, kb * BKB, row_b);
+          tma_load_2d_pair(sb + BN_BOX * BKB, &tmB, fb, kb * BKB, row_b + BN_MMA);
+        }
+      }
+      griddep_wait();
+      int nkb_o = -1;  // read when the first outlier K-block is reached
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         int m_blk, n_blk;
         tile_coords(tile, num_m, num_n, m_blk, n_blk);
         const int row_a = m_blk * 2 * BM + static_cast<int>(rank) * BM;
         const int row_b = n_blk * BN + static_cast<int>(rank) * BN_BOX;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&empty_bar[s], ph ^ 1u, &abort_sh, p.st, W_EMPTY)) {
-            ok = false;
-            break;
+        for (int kb = 0;; ++kb) {
+          if (kb >= p.nkb_i8) {
+            if (nkb_o < 0) nkb_o = outlier_kblocks();
+            if (kb >= p.nkb_i8 + nkb_o) break;
           }
           uint8_t* sa = smem + s * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
-          if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * STAGE_BYTES);
           const uint32_t fb = leader_smem_addr(smem_u32(&full_bar[s]));
-          if (kb < p.nkb_i8) {
+          if (tile == pair && kb < pre) {
+            // stage s == kb: armed and its B halves issued before the wait
 #if I8MP_A_EVICT_LAST
             tma_load_2d_pair_hint(sa, &tmA, fb, kb * BKB, row_a, pol_a);
 #else
             tma_load_2d_pair(sa, &tmA, fb, kb * BKB, row_a);
 #endif
-            tma_load_2d_pair(sb, &tmB, fb, kb * BKB, row_b);
-            tma_load_2d_pair(sb + BN_BOX * BKB, &tmB, fb, kb * BKB, row_b + BN_MMA);
           } else {
-            const int ko = kb - p.nkb_i8;
-            tma_load_2d_pair(sa, &tmAo, fb, ko * 64, row_a);
-            tma_load_2d_pair(sb, &tmBo, fb, ko * 64, row_b);
-            tma_load_2d_pair(sb + BN_BOX * BKB, &tmBo, fb, ko * 64, row_b + BN_MMA);
+            if (!mbar_wait(&empty_bar[s], ph ^ 1u, &abort_sh, p.st, W_EMPTY)) {
+              ok = false;
+              break;
+            }
+            if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * STAGE_BYTES);
+            if (kb < p.nkb_i8) {
+#if I8MP_A_EVICT_LAST
+              tma_load_2d_pair_hint(sa, &tmA, fb, kb * BKB, row_a, pol_a);
+#else
+              tma_load_2d_pair(sa, &tmA, fb, kb * BKB, row_a);
+#endif
+              tma_load_2d_pair(sb, &tmB, fb, kb * BKB, row_b);
+              tma_load_2d_pair(sb + BN_BOX * BKB, &tmB, fb, kb * BKB, row_b + BN_MMA);
+            } else {
+              const int ko = kb - p.nkb_i8;
+              tma_load_2d_pair(sa, &tmAo, fb, ko * 64, row_a);
+              tma_load_2d_pair(sb, &tmBo, fb, ko * 64, row_b);
+              tma_load_2d_pair(sb + BN_BOX * BKB, &tmBo, fb, ko * 64, row_b + BN_MMA);
+            }
           }
           ++issued[s];
           if (++s == STAGES) {
@@ -241,6 +275,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (leader only)
     if (leader && lane == 0) {
+      griddep_wait();
+      const int nkb_o = outlier_kblocks();
+      const int nkb = p.nkb_i8 + nkb_o;
+      const bool has_out = nkb_o > 0;  // outlier product accumulated onto the fp32 partial outputs in TMEM
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -297,6 +335,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
+    griddep_wait();
+    const bool has_out = outlier_kblocks() > 0;
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;  // which EPI_COLS-column group of the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
