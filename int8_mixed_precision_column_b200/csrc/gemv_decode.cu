@@ -10,8 +10,7 @@
 // same count (to one) per CTA: a partial last pass runs with fewer weight
 // loads in flight and, measured, costs about as much as a full one.  The 8
 // warps of a CTA split K; each warp multiplies its K-slice of the 16 x K token
-// codes by the 32 weight rows with mma.sync m16n8k32 (s8 x s8 -> s32), and the
-// warps' int32 partial sums are added in shared memory (exact).
+// codes by the 32 weight rows with mma.sync m16n8k32 (s8 x s8 -> s32).
 // Fragment trick: the dot product is a sum over k, so any permutation of k
 // applied to both operands leaves it unchanged.  Thread (g, t) of a warp loads
 // 16 contiguous bytes of weight row g at k0 + 16t and the same 16 bytes of
@@ -20,10 +19,12 @@
 // its first MMA, so 16 x 16 bytes per thread are in flight (measured against
 // two and three K-steps: 9 % faster at one token; the few bytes the compiler
 // spills at the 128-register bound cost less than the shallower pipeline).
+// The warps' int32 partial sums of a pass meet in one 2 KB shared array by
+// shared-memory atomic adds (exact in any order).
 // Epilogue: Y = TE(acc * sA[t] * SCB[j] / 127^2 + sum_o Xo[t,o] * Wo[j,o] + b[j])
 // with Wo[j,o] = TE((CB[j, idx[o]] * SCB[j]) / 127) recomputed from CB; the
-// outlier operands of a 32-row chunk are staged in shared memory, 64 outlier
-// columns at a time.
+// outlier operands of a 32-row chunk are staged in shared memory, DV_OB
+// outlier columns at a time.
 #include "kernels.h"
 
 namespace i8mp {
@@ -33,7 +34,10 @@ constexpr int DV_WARPS = 8;
 constexpr int DV_THREADS = DV_WARPS * 32;
 constexpr int DV_RG = 4;   // 8-row groups per pass (32 rows)
 constexpr int DV_U = 4;    // K-steps (64 B each) loaded before computing
-constexpr int DV_OB = 64;  // outlier columns staged per block
+#ifndef I8MP_DV_OB
+#define I8MP_DV_OB 16
+#endif
+constexpr int DV_OB = I8MP_DV_OB;  // outlier columns staged per block
 constexpr int kPrefetchRows = 16;  // weight rows per CTA pulled into L2 before the wait
 
 
@@ -79,7 +83,10 @@ __device__ __forceinline__ uint4 ld_stream(const int8_t* p) {
 template <typename TE, bool kExtra>
 __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvParams p) {
   using E = Elem<TE>;
-  __shared__ int32_t red[DV_WARPS][DV_RG][32][4];
+  // int32 partial sums of the pass, added by the 8 warps with shared-memory
+  // atomics (exact in any order); each entry is read and cleared by the one
+  // thread that owns its output
+  __shared__ int32_t red[DV_RG][32][4];
   __shared__ float wo_s[DV_RG * 8][DV_OB + 1];
   __shared__ float xo_s[kDecodeMaxT][DV_OB + 1];
   const int warp = threadIdx.x >> 5;
@@ -108,6 +115,8 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
   const int8_t* xa_base = p.Xq + static_cast<int64_t>(g) * p.K + t4 * 16;
   const int8_t* xb_base = p.Xq + static_cast<int64_t>(g + 8) * p.K + t4 * 16;
   const uint4 zero4 = make_uint4(0, 0, 0, 0);
+  for (int e = threadIdx.x; e < DV_RG * 32 * 4; e += DV_THREADS) (&red[0][0][0])[e] = 0;
+  __syncthreads();
 
   for (int64_t g0 = g_begin; g0 < g_end; g0 += DV_RG) {
     int32_t c[DV_RG][4];
@@ -150,7 +159,7 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
     #pragma unroll
     for (int r = 0; r < DV_RG; ++r) {
       #pragma unroll
-      for (int i = 0; i < 4; ++i) red[warp][r][lane][i] = c[r][i];
+      for (int i = 0; i < 4; ++i) atomicAdd(&red[r][lane][i], c[r][i]);
     }
     __syncthreads();
 
@@ -168,10 +177,8 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
       tok[h] = (ln >> 2) + ((i >> 1) << 3);
       jr[h] = r * 8 + (ln & 3) * 2 + (i & 1);
       live[h] = (g0 + r < g_end) && tok[h] < p.T;
-      int32_t s = 0;
-      #pragma unroll
-      for (int w = 0; w < DV_WARPS; ++w) s += red[w][r][ln][i];
-      acc[h] = s;
+      acc[h] = red[r][ln][i];
+      red[r][ln][i] = 0;  // for the next pass (whose adds follow the pass-end barrier)
     }
     // 16-bit product over the outlier columns, DV_OB columns at a time.
     for (int ob = 0; ob < n_out; ob += DV_OB) {
@@ -227,17 +234,26 @@ __global__ void __launch_bounds__(DV_THREADS, 2) gemv_i8_decode_kernel(const DvP
   }
 }
 
-// Prefer L1 to shared memory: 28 % of the unified storage (the 64 KB
-// configuration) still holds the 2 CTAs per SM, and the token codes, re-read
-// from L1 by every pass, then stay there more often.  Measured at BLOOM FFN-up
-// width: 1.2 % faster at T = 1, 2.3 % at T = 16; the largest shared-memory
-// configuration doubled the time.  A hint, set once per device; a failure is
-// cleared and ignored.
+// Prefer L1 to shared memory: the kernel holds 5.3 KB of shared memory, so
+// the 16 KB configuration (a 7 % carveout) still fits 2 CTAs per SM and
+// leaves about 240 KB to L1 for the token codes that every pass re-reads (the
+// two CTAs of an SM read the same ones).  Measured at BLOOM FFN-up width,
+// product kernel in us, against the previous kernel (per-warp partial sums
+// in 16 KB of shared memory, 64 outlier columns staged, 64 KB configuration):
+// 142.2-142.5 against 146.5-146.9 at T = 1, 144.0-144.2 against 148.2-148.3
+// at T = 4, 156.4-156.5 against 157.4-157.9 at T = 16; the same kernel with
+// the 32 KB or 64 KB configuration took 143.2-144.1, 144.6-145.8 and
+// 156.5-156.9.  (With the old kernel, the largest shared-memory
+// configuration had doubled the time.)  A hint, set once per device; a
+// failure is cleared and ignored.
+#ifndef I8MP_DV_CARVE
+#define I8MP_DV_CARVE 7
+#endif
 bool g_carveout_set[64] = {false};
 
 void prefer_l1(int dev) {
   if (dev < 0 || dev >= 64 || g_carveout_set[dev]) return;
-  const int pct = 28;
+  const int pct = I8MP_DV_CARVE;
   bool ok = cudaFuncSetAttribute(gemv_i8_decode_kernel<__half, false>,
                                  cudaFuncAttributePreferredSharedMemoryCarveout, pct) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(gemv_i8_decode_kernel<__half, true>,
