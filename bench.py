@@ -526,13 +526,17 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     barrier(world)
     torch.cuda.synchronize()
     sampler.mark_begin()
+    # With a flush, each step is bracketed by its own events (the flush stays
+    # outside them); without one, steps run back to back between the outer
+    # events only.
     outer[0].record()
     for i in range(nsteps):
         if flush:
             flush_l2()
-        bounds[i][0].record()
+            bounds[i][0].record()
         step()
-        bounds[i][1].record()
+        if flush:
+            bounds[i][1].record()
     outer[1].record()
     torch.cuda.synchronize()
     sampler.mark_end()
@@ -541,8 +545,8 @@ def run_ours(args, rank, world, local_rank) -> dict | None:
     st, where = native.int8_check_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {native.int8_status_string(st)} at {where:#x}")
-    step_ms = [bounds[i][0].elapsed_time(bounds[i][1]) for i in range(nsteps)]
-    total_ms = outer[0].elapsed_time(outer[1]) if not flush else sum(step_ms)
+    total_ms = sum(bounds[i][0].elapsed_time(bounds[i][1]) for i in range(nsteps)) if flush else \
+        outer[0].elapsed_time(outer[1])
     ms_per_step = reduce_max(total_ms / nsteps, world, dev)
 
     for i in range(nstage):
