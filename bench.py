@@ -41,6 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 POPS)
 
 WORKLOADS = {
+    "toy": lambda dev, seed: workloads.toy(seed=seed, device=dev),
     "bloom176b_ffn_up_prefill": lambda dev, seed: workloads.bloom_ffn_up_prefill(8192, seed=seed, device=dev),
     "bloom176b_ffn_up_prefill_T1024": lambda dev, seed: workloads.bloom_ffn_up_prefill(1024, seed=seed, device=dev),
     "llama7b_prefill": lambda dev, seed: workloads.llama7b_prefill(seed=seed, device=dev),
