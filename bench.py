@@ -122,6 +122,17 @@ def barrier(world: int) -> None:
         dist.barrier()
 
 
+def ensure_library(world: int, local_rank: int) -> None:
+    """Build the library if it is stale, on local rank 0 only; the other ranks
+    wait at a barrier and then load the finished file."""
+    from int8_mixed_precision_column_b200 import build, native
+
+    if world == 1 or local_rank == 0:
+        build.build()
+    barrier(world)
+    native.lib()
+
+
 def rank_seed(rank: int) -> int:
     """Each rank draws its own independent problem (weak scaling)."""
     return 1000 * rank
@@ -225,12 +236,11 @@ def run_sharded(args, rank, world, local_rank) -> dict | None:
     """One layer split along N over the ranks (strong scaling: the total work
     is the one layer), Y assembled on every rank by the product kernels'
     stores into every rank's symmetric output buffer."""
-    from int8_mixed_precision_column_b200 import build, native, sharded
+    from int8_mixed_precision_column_b200 import native, sharded
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    build.build()
-    native.lib()
+    ensure_library(world, local_rank)
     p = WORKLOADS[args.workload]("cuda", rank_seed(0))  # the same layer and batch on every rank
     if args.threshold is not None:
         p.threshold = args.threshold
@@ -455,12 +465,11 @@ def run_decode_lines(args, rank, world, dev) -> dict:
 
 
 def run_ours(args, rank, world, local_rank) -> dict | None:
-    from int8_mixed_precision_column_b200 import build, native
+    from int8_mixed_precision_column_b200 import native
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    build.build()
-    native.lib()
+    ensure_library(world, local_rank)
     p = WORKLOADS[args.workload]("cuda", rank_seed(rank))
     if args.threshold is not None:
         p.threshold = args.threshold

@@ -1,8 +1,11 @@
 """Build libint8mp.so (the CUDA kernels + C ABI) in-tree for sm_100a.
 
 Usage: ``python -m int8_mixed_precision_column_b200.build [--force] [-v]``.
-Each ``csrc/*.cu`` is compiled to an object under ``_build/`` (in parallel),
-then linked into ``int8_mixed_precision_column_b200/lib/libint8mp.so``.
+Each ``csrc/*.cu`` is compiled to an object under ``_build/<pid>/`` (in
+parallel), then linked into a temporary file that atomically replaces
+``int8_mixed_precision_column_b200/lib/libint8mp.so``: processes that build
+at the same time (the ranks of a multi-GPU run) never read each other's
+partial objects, and a process loading the library sees a complete file.
 No fast-math: the quantisation stages must round exactly like IEEE fp32.
 """
 
@@ -46,8 +49,8 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, outdir: str, verbose: bool) -> str:
+    obj = os.path.join(outdir, os.path.basename(src)[:-3] + ".o")
     cmd = [nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
     if verbose:
         cmd += ["-Xptxas", "-v"]
@@ -62,17 +65,23 @@ def _compile(src: str, verbose: bool) -> str:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    outdir = os.path.join(BUILD, str(os.getpid()))
+    os.makedirs(outdir, exist_ok=True)
     os.makedirs(os.path.dirname(LIB), exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
+    tmp = f"{LIB}.{os.getpid()}.tmp"
+    try:
+        with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
+            objs = list(ex.map(lambda s: _compile(s, outdir, verbose), srcs))
+        cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+        os.replace(tmp, LIB)
+    finally:
+        shutil.rmtree(outdir, ignore_errors=True)
+        if os.path.exists(tmp):
+            os.remove(tmp)
     return LIB
 
 
