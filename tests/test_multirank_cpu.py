@@ -35,6 +35,8 @@ def _rank_main(rank: int, world: int, port: int, outdir: str) -> None:
     try:
         r, w, lr = bench.dist_env()
         assert (r, w, lr) == (rank, world, rank)
+        # local rank 0 builds the library if stale; every rank loads it after the barrier
+        bench.ensure_library(world, lr)
         p = workloads.make_problem("rank", 8, 64, 32, n_planted=2, bias_std=0.01, seed=bench.rank_seed(rank))
         local_ms = 1.0 + 0.5 * rank          # rank 1 is the slow one
         bench.barrier(world)
